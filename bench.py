@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark: VideoMLA latent-KV chunk attention on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 480p]
+
+One step = one pass of the hot path over one chunk of the 480P workload
+(Wan2.1-1.3B shape: 30 x 52 patches per frame, a chunk of 3 frames = 4680
+queries, a 21-frame window = 32760 keys, 12 heads x 128, d_c = 192, d_r = 32):
+    vmla_cache_append     the chunk's 4680 tokens -> [c ; RoPE3D(k_r)] rows of the window
+    vmla_chunk_attention  4680 queries x 12 heads over the 32760 cached keys
+Inputs are seeded synthetic data (see the `workload` package) already resident in
+HBM when the timed region starts; L2 is flushed (256 MiB write) before every timed
+step.  `value` counts the absorbed-MLA tensor FLOPs of the attention,
+2*B*Nq*H*Nkv*(224+192), plus the append's 2*B*Nq*224*1536, per second.  The dense
+per-head baseline (3072 scalars/token) is timed on the same queries beside it.
+
+Under torchrun (N > 1) every rank runs an independent replica on its own seed
+(no data-path collective); the time is the max over ranks and `value` the work of
+all ranks over that time.  --impl reference times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workload  # noqa: E402
+
+METRIC = "MLA chunk-attention TFLOP/s & ms/chunk (Wan-1.3B 480P shape); % BF16 peak"
+UNIT = "TFLOP/s"
+SCALE = 160 ** -0.5
+FLUSH_BYTES = 256 << 20
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "chunk_attn_480p_ncu.md")
+ATTN_SOURCES = [os.path.join(ROOT, "latent_kv_cache_b200", "csrc", f)
+                for f in ("attention.cu", "sm100.cuh", "common.cuh")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="480p", choices=sorted(workload.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def workload_desc(w) -> dict:
+    return {
+        "workload": (f"{w.name}: B={w.batch}, {w.grid_h}x{w.grid_w} patches/frame, chunk {w.chunk_frames} "
+                     f"frames = {w.n_q} queries, window {w.window_frames} frames = {w.n_kv} keys "
+                     f"({w.cached_frames} cached + chunk), H={w.heads}x{w.d_head}, d_c={w.d_c}, d_r={w.d_r}"),
+        "batch": w.batch, "n_q": w.n_q, "n_kv": w.n_kv, "heads": w.heads, "d_c": w.d_c, "d_r": w.d_r,
+        "step": "cache_append(chunk) + chunk_attention(window)",
+        "l2": "flushed before every timed step (256 MiB write)",
+        "flops_convention": "absorbed MLA: 2*B*Nq*H*Nkv*(d_c+d_r+d_c) + append 2*B*Nq*224*1536",
+    }
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0.0)), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in ATTN_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    or None if the summary is missing or the kernel source changed since."""
+    try:
+        vals = {}
+        with open(PROFILE_SUMMARY) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    vals[k.strip()] = v.strip().strip("`")
+        if vals.get("source_sha256_16") != attn_source_hash():
+            return None
+        return int(vals["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML; falls back to nvidia-smi)
+# ---------------------------------------------------------------------------
+_REASONS = [(0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+            (0x2, "applications_clocks_setting"), (0x10, "sync_boost")]
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._dev = device_index
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _reasons_now(self):
+        n = self._nvml
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(n, fn):
+                try:
+                    return int(getattr(n, fn)(self._h))
+                except Exception:
+                    pass
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                self.reasons |= self._reasons_now()
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self) -> dict:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [name for bit, name in _REASONS if self.reasons & bit]}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle as it stands, on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(d.get("num_threads", 1)) for d in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(w, act, wts, cache_bits, rows, n_tok):
+    """One bounded oracle step: append of n_tok chunk tokens + attention of `rows` queries."""
+    import oracle
+    x_tok = act["x"][:, w.n_cached:w.n_cached + n_tok]
+    t0 = time.perf_counter()
+    oracle.cache_append(x_tok, wts["w_dkv"], wts["w_kr"], w.chunk_t0, w.grid_h, w.grid_w)
+    oracle.chunk_attention(act["q"], act["q_rope"], wts["w_uk"], wts["w_uv"], cache_bits, w.n_kv,
+                           w.chunk_t0, w.grid_h, w.grid_w, SCALE, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = (w.attention_flops() * len(rows) / w.n_q + w.append_flops(n_tok))
+    return dt, flops
+
+
+def oracle_prepare(w, act, wts):
+    import oracle
+    return oracle.cache_append(act["x"], wts["w_dkv"], wts["w_kr"], 0, w.grid_h, w.grid_w)
+
+
+def size_oracle_sample(w, act, wts, cache_bits, target_s):
+    """Rows/tokens of one oracle step taking about target_s seconds."""
+    rows = np.arange(0, w.n_q, max(1, w.n_q // 32))[:32]
+    dt, _ = oracle_sample_step(w, act, wts, cache_bits, rows, 64)
+    per = max(dt, 1e-3)
+    scale = max(1.0, target_s / per)
+    n_rows = int(min(w.n_q, max(8, 32 * scale)))
+    n_tok = int(min(w.n_q, max(32, 64 * scale)))
+    return np.linspace(0, w.n_q - 1, n_rows).astype(np.int64), n_tok
+
+
+def cpu_baseline(w, act, wts, target_s):
+    cache_bits = oracle_prepare(w, act, wts)
+    rows, n_tok = size_oracle_sample(w, act, wts, cache_bits, target_s)
+    dt, flops = oracle_sample_step(w, act, wts, cache_bits, rows, n_tok)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": (f"fp64 oracle: append of {n_tok} chunk tokens + attention of {len(rows)} of "
+                       f"{w.n_q} query rows x {w.heads} heads x {w.n_kv} keys; {dt:.1f} s; FLOPs "
+                       f"counted with the same absorbed convention as the GPU value"),
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the oracle timed on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    wts = workload.layer_weights(w)
+    act = workload.batch_activations(w)
+    cache_bits = oracle_prepare(w, act, wts)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows, n_tok = size_oracle_sample(w, act, wts, cache_bits, min(2.0, budget))
+    for _ in range(args.warmup):
+        oracle_sample_step(w, act, wts, cache_bits, rows, n_tok)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_step(w, act, wts, cache_bits, rows, n_tok)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"fp64 oracle per step: append of {n_tok} chunk tokens + attention of {len(rows)} of "
+              f"{w.n_q} query rows x {w.heads} heads x {w.n_kv} keys")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_desc(w), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": _blas_threads(),
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import latent_kv_cache_b200 as vm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # Each rank is an independent replica with its own seed (weak scaling).
+    wr = w.with_(seed=w.seed + 100003 * rank)
+    wts = workload.layer_weights(wr)
+    act = workload.batch_activations(wr)
+
+    def T(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x_all = T(act["x"])
+    wd, wk, wuk, wuv = T(wts["w_dkv"]), T(wts["w_kr"]), T(wts["w_uk"]), T(wts["w_uv"])
+    q, qr = T(act["q"]), T(act["q_rope"])
+    out = torch.empty_like(q)
+    cache = torch.zeros(w.batch, w.n_kv, 224, dtype=torch.bfloat16, device=dev)
+    per = w.tokens_per_frame
+    for f0 in range(0, w.cached_frames, w.chunk_frames):  # the window's cached frames
+        nf = min(w.chunk_frames, w.cached_frames - f0)
+        vm.vmla_cache_append(x_all[:, f0 * per:(f0 + nf) * per].contiguous(), wd, wk, cache, f0 * per, f0,
+                             w.grid_h, w.grid_w)
+    x_chunk = x_all[:, w.n_cached:].contiguous()
+    del x_all
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        vm.vmla_cache_append(x_chunk, wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w, stream)
+        vm.vmla_chunk_attention(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                out, stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step()
+    vm.vmla_get_device_status(stream)
+
+    # ---- timed region: K steps, L2 flushed before each, events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    sampler.start()
+    for k in range(args.steps):
+        flush_buf.zero_()
+        ev[k][0].record(stream)
+        vm.vmla_cache_append(x_chunk, wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w, stream)
+        ev[k][1].record(stream)
+        vm.vmla_chunk_attention(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                out, stream)
+        ev[k][2].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    vm.vmla_get_device_status(stream)
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    app_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(step_ms))
+    gpu_launches = 2 * args.steps
+
+    flops_step = w.attention_flops() + w.append_flops()
+    value = world * args.steps * flops_step / (total_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / args.steps
+    attn_mean = sum(attn_ms) / len(attn_ms)
+    app_mean = sum(app_ms) / len(app_ms)
+
+    # ---- dense per-head baseline on the same queries (3072 scalars per token)
+    kv = workload.batch_dense_kv(wr)
+    kd, vd = T(kv["k"]), T(kv["v"])
+    out_d = torch.empty_like(q)
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        vm.vmla_dense_attention(q, kd, vd, SCALE, out_d, stream)
+    dense_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush_buf.zero_()
+        dense_ev[k][0].record(stream)
+        vm.vmla_dense_attention(q, kd, vd, SCALE, out_d, stream)
+        dense_ev[k][1].record(stream)
+    barrier()
+    vm.vmla_get_device_status(stream)
+    dense_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in dense_ev)) / args.steps
+    del kd, vd, out_d
+
+    # ---- end to end through the public API: pinned host inputs -> device -> host result
+    h_x = x_chunk.cpu().pin_memory()
+    h_q = q.cpu().pin_memory()
+    h_qr = qr.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = h_x.numel() * 2 + h_q.numel() * 2 + h_qr.numel() * 2
+    d2h = h_out.numel() * 2
+
+    def e2e_step():
+        x_chunk.copy_(h_x, non_blocking=True)
+        q.copy_(h_q, non_blocking=True)
+        qr.copy_(h_qr, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        e2e_step()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush_buf.zero_()
+        e2e_ev[k][0].record(stream)
+        e2e_step()
+        e2e_ev[k][1].record(stream)
+    barrier()
+    vm.vmla_get_device_status(stream)
+    e2e_total = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev))
+    e2e_value = world * args.steps * flops_step / (e2e_total * 1e-3) / 1e12
+
+    peak, peak_sust, hbm, peak_src = measured_peaks()
+    achieved = w.attention_flops() / (attn_mean * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_desc(w),
+        "ms_chunk_attention": attn_mean, "ms_cache_append": app_mean,
+        "attention_tflops": achieved,
+        "pct_bf16_peak": 100.0 * achieved / peak,
+        "pct_bf16_peak_sustained": 100.0 * achieved / peak_sust if peak_sust else None,
+        "pct_bf16_nominal_2250": 100.0 * achieved / 2250.0,
+        "attention_layer_tokens_per_s": w.batch * w.n_q / (attn_mean * 1e-3),
+        "dense": {"ms": dense_ms, "tflops": w.dense_flops() / (dense_ms * 1e-3) / 1e12,
+                  "mla_over_dense_ms": attn_mean / dense_ms,
+                  "cache_bytes_per_token": {"mla": 224 * 2, "dense": 3072 * 2}},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "kernel": "k_chunk_attn"},
+        "append": {"us": app_mean * 1e3, "bound": "alu",
+                   "gbs": (x_chunk.numel() * 2 + 224 * w.d_model * 2 + w.batch * w.n_q * 224 * 2)
+                   / (app_mean * 1e-3) / 1e9, "hbm_peak_gbs": hbm},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_total / args.steps},
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, act, wts, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workload.CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    return run_ours(args, w, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * videomla.h -- C ABI of the B200 (sm_100a) VideoMLA latent-KV chunk-attention library.
+ *
+ * Method: VideoMLA, "Low-Rank Latent KV Cache for Minute-Scale Autoregressive
+ * Video Diffusion" (abstract; summary page, "Approach" and "Key results").
+ * In chunk-causal autoregressive video diffusion (Wan2.1-T2V-1.3B, 12 heads of
+ * 128) every cached token keeps, per layer, a head-shared content latent
+ * c = x . W_DKV^T (d_c = 192) and a head-shared decoupled 3D-RoPE key
+ * k_r = RoPE3D(x . W_KR^T) (d_r = 32): 224 scalars instead of 2 x 12 x 128 = 3072
+ * (92.7% less).  The current chunk's queries attend to the sliding window of
+ * cached frames plus the chunk itself.
+ *
+ * Conventions for every call
+ *   - bf16 data are passed as pointers to their 16-bit patterns (uint16_t).
+ *   - All tensor pointers are DEVICE pointers, contiguous row-major, 16-byte
+ *     aligned.  The caller owns every buffer; the library allocates no device
+ *     memory per call.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it and never synchronise, except vmla_get_device_status.
+ *   - Argument errors return VMLA_ERR_INVALID_ARG / VMLA_ERR_UNSUPPORTED before
+ *     anything is launched; no output is written then.  vmla_last_error()
+ *     describes the most recent failure of the calling thread.
+ *   - Kernels never trap.  Every internal wait has a time limit; a wait that
+ *     runs out records a code that vmla_get_device_status reports.
+ *   - Compiled sizes: d_c = 192, d_r = 32, per-head dim 128.  The 32 rope dims
+ *     split into (t: 12, h: 10, w: 10); pair i of an axis with d_a dims turns at
+ *     1e4^(-2i/d_a) radians per position; pairs are adjacent dims.
+ *   - Token n of a call that starts at frame t0 on a grid_h x grid_w patch grid
+ *     sits at (t0 + n / (grid_h*grid_w), (n / grid_w) % grid_h, n % grid_w);
+ *     grid_h, grid_w <= 256 and a call spans at most 32 frames.
+ */
+#ifndef VIDEOMLA_H
+#define VIDEOMLA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VMLA_OK = 0,
+  VMLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size */
+  VMLA_ERR_UNSUPPORTED = 2, /* size outside what the kernels are compiled for */
+  VMLA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  VMLA_ERR_TIMEOUT = 4      /* a kernel wait ran out of time (reported by vmla_get_device_status) */
+} vmla_status;
+
+/* Human-readable name of a status code (static string). */
+const char* vmla_status_string(int status);
+
+/* Description of the last error returned to the calling thread (static per thread). */
+const char* vmla_last_error(void);
+
+/*
+ * vmla_cache_append -- down-projection, 3D-RoPE and write into the latent cache.
+ * (abstract: "shared low-rank content latent and a shared decoupled 3D-RoPE
+ * positional key"; summary "Approach"; summary "Key results": 224 scalars.)
+ *
+ *   x      [batch, n_tok, d_model]   bf16, hidden states of the new tokens
+ *   w_dkv  [192, d_model]            bf16, nn.Linear layout [out, in]
+ *   w_kr   [32, d_model]             bf16
+ *   cache  [batch, cap, 224]         bf16, row = [c (192) ; rotated k_r (32)]
+ *
+ * Token n of sample b goes to cache row (slot0 + n) mod cap of sample b (the
+ * sliding window is a ring of `cap` slots; attention does not depend on slot
+ * order).  Each output value is computed in fp32 with the fixed order
+ *   acc = 0; for k = 0..d_model-1: acc = fl(acc + x[k]*w[k])   (exact products),
+ * then, for the rope pairs (a, b): a' = fl(fl(a*cos) - fl(b*sin)),
+ * b' = fl(fl(a*sin) + fl(b*cos)) with cos/sin the fp32 roundings of the fp64 libm
+ * values, then rounded to bf16 (nearest even) -- so results are reproducible bit
+ * for bit on any device.
+ * Limits: d_model a multiple of 64 in [64, 16384]; 1 <= n_tok <= cap;
+ * 0 <= slot0 < cap; t0 >= 0.
+ */
+vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                              int32_t batch, int32_t n_tok, int32_t d_model, uint16_t* cache,
+                              int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
+                              int32_t grid_w, void* stream);
+
+/*
+ * vmla_chunk_attention -- multi-head latent attention of one chunk over the cache.
+ * (abstract and summary "Approach": per-head keys/values replaced by the shared
+ * latent and rope key; summary: chunk-causal AR video diffusion.)
+ *
+ *   q      [batch, n_q, heads, 128]  bf16, content queries of the chunk
+ *   q_rope [batch, n_q, heads, 32]   bf16, rope queries, NOT yet rotated; query i is
+ *                                    rotated with the position of token i of a chunk
+ *                                    starting at frame t0
+ *   w_uk   [heads*128, 192]          bf16, key up-projection (row h*128+d)
+ *   w_uv   [heads*128, 192]          bf16, value up-projection (row h*128+e)
+ *   cache  [batch, cap, 224]         bf16, keys are rows [0, n_kv)
+ *   out    [batch, n_q, heads, 128]  bf16
+ *
+ * Computes, for every sample b, head h and query i,
+ *   out[b,i,h,:] = softmax_j( scale * ( q_h,i . W_UK_h . c_j + RoPE(q_r,h,i) . k_r,j ) )
+ *                  . (c_j . W_UV_h^T)                     over all keys j in [0, n_kv)
+ * i.e. every query sees every cached key and every key of its own chunk
+ * (bidirectional inside the chunk).  W_UK is absorbed into the queries and
+ * W_UV is applied once per query after the latent accumulation; bf16 tensor-core
+ * products with fp32 accumulation.
+ * Limits: 1 <= n_kv <= cap < 2^31; n_q >= 1; heads >= 1; scale > 0 and finite.
+ */
+vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                 const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                 int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv,
+                                 int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
+                                 uint16_t* out, void* stream);
+
+/*
+ * vmla_dense_attention -- the per-head (3072-scalar) baseline layout, for comparison.
+ * (summary "Key results": Self-Forcing's dense per-head KV cache, 3072 scalars/token.)
+ *
+ *   q    [batch, n_q, heads, d_head]   bf16
+ *   k, v [batch, n_kv, heads, d_head]  bf16 (rope already applied to k)
+ *   out  [batch, n_q, heads, d_head]   bf16
+ * out[b,i,h,:] = softmax_j(scale * q_h,i . k_h,j) . v_h,j over j in [0, n_kv).
+ * Limits: d_head == 128; n_kv >= 1; n_q >= 1; heads >= 1.
+ */
+vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 int32_t batch, int32_t n_q, int64_t n_kv, int32_t heads,
+                                 int32_t d_head, float scale, uint16_t* out, void* stream);
+
+/*
+ * vmla_get_device_status -- synchronises `stream`, then reports (and clears) any
+ * wait timeout recorded by this library's kernels on the current device since the
+ * last call: VMLA_ERR_TIMEOUT, VMLA_ERR_CUDA on a CUDA error, else VMLA_OK.
+ */
+vmla_status vmla_get_device_status(void* stream);
+
+/*
+ * vmla_selftest_wait_timeout -- launches one tiny kernel that waits on a barrier
+ * nothing will ever complete, with a limit of `limit_ns` nanoseconds (1e3 .. 1e10).
+ * The kernel gives up, records a timeout and returns, leaving the context usable;
+ * a following vmla_get_device_status(stream) returns VMLA_ERR_TIMEOUT.  For tests
+ * of the failure path.
+ */
+vmla_status vmla_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VIDEOMLA_H */

@@ -1,0 +1,174 @@
+// C ABI of the library (declared in include/videomla.h): argument validation,
+// error reporting and dispatch to the kernels.  Nothing here allocates device
+// memory; every tensor belongs to the caller.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "common.cuh"
+#include "videomla.h"
+
+namespace vmla {
+cudaError_t launch_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                                int batch, int n_tok, int d_model, uint16_t* cache, int64_t cap,
+                                int64_t slot0, int64_t t0, int grid_h, int grid_w, cudaStream_t stream);
+cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                   const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
+                                   int heads, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
+                                   int grid_w, float scale, uint16_t* out, int* status,
+                                   cudaStream_t stream, bool* encode_failed);
+cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int batch,
+                                   int n_q, int64_t n_kv, int heads, float scale, uint16_t* out,
+                                   int* status, cudaStream_t stream, bool* encode_failed);
+cudaError_t launch_selftest_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t s);
+}  // namespace vmla
+
+namespace {
+
+thread_local char g_last_error[512] = "no error";
+
+vmla_status fail(vmla_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vmla_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(VMLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Common checks of the rotary-position arguments of a call covering n_tok tokens.
+vmla_status check_positions(int64_t n_tok, int64_t t0, int32_t grid_h, int32_t grid_w) {
+  if (grid_h < 1 || grid_w < 1) return fail(VMLA_ERR_INVALID_ARG, "grid_h/grid_w must be >= 1");
+  if (grid_h > vmla::kMaxSide || grid_w > vmla::kMaxSide)
+    return fail(VMLA_ERR_UNSUPPORTED, "grid_h/grid_w must be <= %d", vmla::kMaxSide);
+  if (t0 < 0) return fail(VMLA_ERR_INVALID_ARG, "t0 must be >= 0");
+  const int64_t per = (int64_t)grid_h * grid_w;
+  if ((n_tok + per - 1) / per > vmla::kMaxFrames)
+    return fail(VMLA_ERR_UNSUPPORTED, "a call may span at most %d frames", vmla::kMaxFrames);
+  return VMLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vmla_status_string(int status) {
+  switch (status) {
+    case VMLA_OK: return "VMLA_OK";
+    case VMLA_ERR_INVALID_ARG: return "VMLA_ERR_INVALID_ARG";
+    case VMLA_ERR_UNSUPPORTED: return "VMLA_ERR_UNSUPPORTED";
+    case VMLA_ERR_CUDA: return "VMLA_ERR_CUDA";
+    case VMLA_ERR_TIMEOUT: return "VMLA_ERR_TIMEOUT";
+    default: return "VMLA_ERR_UNKNOWN";
+  }
+}
+
+const char* vmla_last_error(void) { return g_last_error; }
+
+vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                              int32_t batch, int32_t n_tok, int32_t d_model, uint16_t* cache,
+                              int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
+                              int32_t grid_w, void* stream) {
+  if (!aligned16(x) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(cache))
+    return fail(VMLA_ERR_INVALID_ARG, "cache_append: pointers must be non-null and 16-byte aligned");
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "cache_append: batch must be in [1, 65535]");
+  if (n_tok < 1) return fail(VMLA_ERR_INVALID_ARG, "cache_append: n_tok must be >= 1");
+  if (d_model < 64 || d_model > 16384 || d_model % 64 != 0)
+    return fail(VMLA_ERR_UNSUPPORTED, "cache_append: d_model must be a multiple of 64 in [64, 16384]");
+  if (cap < 1 || n_tok > cap) return fail(VMLA_ERR_INVALID_ARG, "cache_append: need 1 <= n_tok <= cap");
+  if (slot0 < 0 || slot0 >= cap) return fail(VMLA_ERR_INVALID_ARG, "cache_append: need 0 <= slot0 < cap");
+  vmla_status st = check_positions(n_tok, t0, grid_h, grid_w);
+  if (st != VMLA_OK) return st;
+  cudaError_t e = vmla::launch_cache_append(x, w_dkv, w_kr, batch, n_tok, d_model, cache, cap, slot0,
+                                            t0, grid_h, grid_w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cache_append launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                 const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                 int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv,
+                                 int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
+                                 uint16_t* out, void* stream) {
+  if (!aligned16(q) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(w_uv) ||
+      !aligned16(cache) || !aligned16(out))
+    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: pointers must be non-null and 16-byte aligned");
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: batch must be in [1, 65535]");
+  if (n_q < 1) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: n_q must be >= 1");
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: heads must be in [1, 512]");
+  if (n_kv < 1 || n_kv > cap) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: need 1 <= n_kv <= cap");
+  if (cap >= (int64_t(1) << 31)) return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: cap must be < 2^31");
+  if ((int64_t)((n_q + 127) / 128) * heads > 0x7FFFFFFF)
+    return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: too many query tiles");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: scale must be positive and finite");
+  vmla_status st = check_positions(n_q, t0, grid_h, grid_w);
+  if (st != VMLA_OK) return st;
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "chunk_attention: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_chunk_attention(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap,
+                                               n_kv, t0, grid_h, grid_w, scale, out, status,
+                                               static_cast<cudaStream_t>(stream), &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "chunk_attention: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 int32_t batch, int32_t n_q, int64_t n_kv, int32_t heads,
+                                 int32_t d_head, float scale, uint16_t* out, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(VMLA_ERR_INVALID_ARG, "dense_attention: pointers must be non-null and 16-byte aligned");
+  if (d_head != vmla::kDh) return fail(VMLA_ERR_UNSUPPORTED, "dense_attention: d_head must be 128");
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "dense_attention: batch must be in [1, 65535]");
+  if (n_q < 1) return fail(VMLA_ERR_INVALID_ARG, "dense_attention: n_q must be >= 1");
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "dense_attention: heads must be in [1, 512]");
+  if (n_kv < 1 || n_kv >= (int64_t(1) << 31))
+    return fail(VMLA_ERR_INVALID_ARG, "dense_attention: need 1 <= n_kv < 2^31");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VMLA_ERR_INVALID_ARG, "dense_attention: scale must be positive and finite");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "dense_attention: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_dense_attention(q, k, v, batch, n_q, n_kv, heads, scale, out, status,
+                                               static_cast<cudaStream_t>(stream), &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "dense_attention: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "dense_attention launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_get_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "get_device_status: stream synchronize");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "get_device_status: no CUDA device");
+  int code = 0;
+  e = cudaMemcpy(&code, status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "get_device_status: read status");
+  if (code != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "get_device_status: clear status");
+    return fail(VMLA_ERR_TIMEOUT, "a kernel wait ran out of time (device code %d)", code);
+  }
+  return VMLA_OK;
+}
+
+vmla_status vmla_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll)
+    return fail(VMLA_ERR_INVALID_ARG, "selftest_wait_timeout: limit_ns must be in [1e3, 1e10]");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "selftest_wait_timeout: no CUDA device");
+  cudaError_t e = vmla::launch_selftest_wait_timeout(status, (uint64_t)limit_ns,
+                                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_timeout launch");
+  return VMLA_OK;
+}
+
+}  // extern "C"

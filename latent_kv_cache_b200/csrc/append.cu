@@ -1,0 +1,184 @@
+// Latent-cache append: c = x . W_DKV^T, k_r = RoPE3D(x . W_KR^T), 16-byte row writes.
+//
+// VideoMLA ("Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video
+// Diffusion", abstract and summary "Approach"): each cached token stores a
+// head-shared content latent (192) and a head-shared decoupled 3D-RoPE key (32).
+//
+// The arithmetic order is fixed so the result is reproducible bit for bit:
+// every output is one fp32 accumulator updated for k = 0, 1, ..., d_model-1
+// with fma(x_k, w_k, acc) -- bf16 x bf16 products are exact in fp32, so each step
+// equals fl(acc + x_k w_k) -- then the rope pairs are rotated with separately
+// rounded products and sums (__fmul_rn / __fadd_rn / __fsub_rn, no contraction),
+// then rounded to bf16 (nearest even).  This is CUDA-core work: the tensor
+// cores do not specify their accumulation order.
+//
+// Tiling: a CTA owns 32 tokens x all 224 outputs; each of its 4 warps owns 8
+// tokens, and lane l owns outputs l + 32 i (i = 0..6), so the rope dims (outputs
+// 192..223) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
+// Operands are staged per 64-wide k chunk in shared memory as fp32.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace vmla {
+
+namespace {
+constexpr int kTok = 32;         // tokens per CTA
+constexpr int kKc = 64;          // k chunk
+constexpr int kThreads = 128;    // 4 warps
+constexpr int kTokPerWarp = 8;
+constexpr int kOutPerLane = 7;   // 224 / 32
+constexpr int kStride = kKc + 4; // fp32 row stride in shared memory (conflict-free float4 reads)
+constexpr int kSmemBytes = (kDrow + kTok) * kStride * 4;
+
+struct AppendParams {
+  const uint16_t* x;
+  const uint16_t* w_dkv;
+  const uint16_t* w_kr;
+  uint16_t* cache;
+  int64_t cap;
+  int64_t slot0;
+  int n_tok;
+  int d_model;
+  int grid_h;
+  int grid_w;
+};
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float4& lo, float4& hi) {
+  lo = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+  hi = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_cache_append(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
+  extern __shared__ __align__(16) float smem_f[];
+  float* ws = smem_f;                   // [224][kStride]  weights of the chunk
+  float* xs = smem_f + kDrow * kStride; // [32][kStride]   tokens of the chunk
+  const int b = blockIdx.y;
+  const int tok0 = blockIdx.x * kTok;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* xb = p.x + (int64_t)b * p.n_tok * p.d_model;
+
+  float acc[kTokPerWarp][kOutPerLane];
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+    for (int i = 0; i < kOutPerLane; ++i) acc[t][i] = 0.0f;
+
+  for (int k0 = 0; k0 < p.d_model; k0 += kKc) {
+    __syncthreads();
+    for (int v = threadIdx.x; v < kDrow * 8; v += kThreads) {
+      const int n = v >> 3, kk = (v & 7) * 8;
+      const uint16_t* src = n < kDc ? p.w_dkv + (int64_t)n * p.d_model
+                                    : p.w_kr + (int64_t)(n - kDc) * p.d_model;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + k0 + kk));
+      float4 lo, hi;
+      bf16x8_to_f32(u, lo, hi);
+      *reinterpret_cast<float4*>(ws + n * kStride + kk) = lo;
+      *reinterpret_cast<float4*>(ws + n * kStride + kk + 4) = hi;
+    }
+    for (int v = threadIdx.x; v < kTok * 8; v += kThreads) {
+      const int t = v >> 3, kk = (v & 7) * 8;
+      float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+      if (tok0 + t < p.n_tok) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)(tok0 + t) * p.d_model + k0 + kk));
+        bf16x8_to_f32(u, lo, hi);
+      }
+      *reinterpret_cast<float4*>(xs + t * kStride + kk) = lo;
+      *reinterpret_cast<float4*>(xs + t * kStride + kk + 4) = hi;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int kk = 0; kk < kKc; kk += 4) {
+      float4 wv[kOutPerLane];
+#pragma unroll
+      for (int i = 0; i < kOutPerLane; ++i)
+        wv[i] = *reinterpret_cast<const float4*>(ws + (lane + 32 * i) * kStride + kk);
+#pragma unroll
+      for (int t = 0; t < kTokPerWarp; ++t) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + (warp * kTokPerWarp + t) * kStride + kk);
+#pragma unroll
+        for (int i = 0; i < kOutPerLane; ++i) {
+          float a = acc[t][i];
+          a = fmaf(xv.x, wv[i].x, a);  // k
+          a = fmaf(xv.y, wv[i].y, a);  // k + 1
+          a = fmaf(xv.z, wv[i].z, a);  // k + 2
+          a = fmaf(xv.w, wv[i].w, a);  // k + 3
+          acc[t][i] = a;
+        }
+      }
+    }
+  }
+
+  // 3D rotary embedding of the rope dims (output 192 + lane).
+  const int pair = lane >> 1;
+  const bool even = (lane & 1) == 0;
+  const int per_frame = p.grid_h * p.grid_w;
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t) {
+    const int tok = tok0 + warp * kTokPerWarp + t;
+    const float v = acc[t][6];
+    const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+    if (tok < p.n_tok) {
+      const int f = tok / per_frame;
+      const int rem = tok - f * per_frame;
+      const int row = rem / p.grid_w;
+      const int col = rem - row * p.grid_w;
+      float2 cs;
+      if (pair < kPairsT) cs = tab.t[f][pair];
+      else if (pair < kPairsT + kPairsH) cs = tab.h[row][pair - kPairsT];
+      else cs = tab.w[col][pair - kPairsT - kPairsH];
+      const float a = even ? v : other;
+      const float bb = even ? other : v;
+      acc[t][6] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
+                       : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
+    }
+  }
+
+  // Stage the 32 x 224 bf16 rows in shared memory, then write 16-byte vectors.
+  __syncthreads();
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_f);
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+    for (int i = 0; i < kOutPerLane; ++i)
+      os[(warp * kTokPerWarp + t) * kDrow + lane + 32 * i] = __float2bfloat16_rn(acc[t][i]);
+  __syncthreads();
+  constexpr int kVecPerRow = kDrow * 2 / 16;  // 28
+  for (int v = threadIdx.x; v < kTok * kVecPerRow; v += kThreads) {
+    const int t = v / kVecPerRow, c = v - t * kVecPerRow;
+    const int tok = tok0 + t;
+    if (tok < p.n_tok) {
+      const int64_t slot = (p.slot0 + tok) % p.cap;
+      uint4 val = *reinterpret_cast<const uint4*>(os + t * kDrow + c * 8);
+      *reinterpret_cast<uint4*>(p.cache + ((int64_t)b * p.cap + slot) * kDrow + c * 8) = val;
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                                int batch, int n_tok, int d_model, uint16_t* cache, int64_t cap,
+                                int64_t slot0, int64_t t0, int grid_h, int grid_w,
+                                cudaStream_t stream) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_cache_append, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  AppendParams p{x, w_dkv, w_kr, cache, cap, slot0, n_tok, d_model, grid_h, grid_w};
+  static thread_local RopeTable tab;
+  const int per_frame = grid_h * grid_w;
+  build_rope_table(&tab, t0, (n_tok + per_frame - 1) / per_frame, grid_h, grid_w);
+  dim3 grid((n_tok + kTok - 1) / kTok, batch);
+  k_cache_append<<<grid, kThreads, kSmemBytes, stream>>>(p, tab);
+  return cudaGetLastError();
+}
+
+}  // namespace vmla
