@@ -11,21 +11,31 @@
 //
 // One CTA = one 128-query tile of one head of one sample; heads are the fastest
 // grid index so the 12 CTAs that read the same cache tiles run together and
-// share them through L2.  Warp roles (192 threads):
-//   warp 0      TMA producer: q tile + W_UK_h, then [c ; k_r] tiles of 128 keys
-//               into a 3-stage ring, then W_UV_h.
+// share them through L2.  Warp roles (320 threads):
+//   warp 0      TMA producer: prologue operands, then key tiles into a ring.
 //   warp 1      TMEM allocation and the single MMA-issuing thread.
-//   warps 2..5  softmax warpgroup; thread = query row = TMEM lane.
-// Tensor memory (512 columns x 128 lanes, fp32):
+//   warps 2..9  two softmax warpgroups; a thread owns one query row (= TMEM
+//               lane) and one half of the columns of every score tile.
+//
+// Shared-memory bandwidth is the budget that sizes this design: the tensor
+// core reads its shared-memory operands and TMA writes the next key tiles
+// through the same ~128 B/clk per SM.  The query operand therefore lives in
+// tensor memory (A operand from TMEM) and only the key tiles come from shared
+// memory: per 96-key MLA tile the tensor core reads 43 KB (K) + 36 KB (V) and
+// TMA writes 43 KB, ~98 B per tensor-core cycle.
+//
+// MLA tensor memory (512 columns x 128 lanes, fp32 cells):
 //   [0,192)   O_lat accumulator (the prologue's q_abs lands here first)
-//   [256,384) S buffer 0   (P, bf16, overwrites its first 64 columns)
-//   [384,512) S buffer 1
-//   epilogue: normalised O_lat as bf16 at [256,352), out accumulator at [384,512).
-// Per key tile j the MMA thread issues S_j = Qa K_j^T (14 MMAs of K=16, the
-// last two over the 64-byte-swizzled rope block) and then O += P_{j-1} C_{j-1}
-// (8 MMAs, P read from tensor memory, C read MN-major from the same smem tile
-// that served as K).  The softmax keeps the running max in log2 units and
-// rescales O only when the max grows by more than 8 (2^8 headroom in bf16 P).
+//   [192,288) S buffer 0 (P, bf16, overwrites its first 48 columns)
+//   [288,384) S buffer 1
+//   [384,496) Qa = [q_abs (96 cells of bf16 pairs) ; rotated q_r (16 cells)]
+//   epilogue: normalised O_lat (bf16) at [192,288), out accumulator at [288,416).
+// Per key tile j the MMA thread issues S_j = Qa K_j^T (14 MMAs, K = 16 each,
+// the last two over the 64-byte-swizzled rope block) and then O += P_{j-1}
+// C_{j-1} (6 MMAs, P read from TMEM, C read MN-major from the same shared-memory
+// tile that served as K: keys and values are one tile).
+// The softmax keeps the running max in log2 units and rescales O only when the
+// max grows by more than 8 (P stays <= 2^8 in bf16).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -35,48 +45,89 @@
 namespace vmla {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kBM = 128;                // queries per tile
-constexpr int kBN = 128;                // keys per tile
-constexpr int kStages = 3;
-constexpr uint32_t kBlk = 16384;        // 128 rows x 128 B (one 128B-swizzled block)
-constexpr uint32_t kMlaStage = 3 * kBlk + 8192;   // [c: 3 blocks | k_r: 128 x 64 B]
-constexpr uint32_t kDenseStage = 4 * kBlk;        // [K: 2 blocks | V: 2 blocks]
-constexpr uint32_t kSmemBarOff = 229376;          // after Qa/Q + 3 stages (both kernels)
-constexpr uint32_t kSmemBytes = kSmemBarOff + 256 + 1024;
-
+constexpr int kSoftmaxWarps = 8;                  // two warpgroups, one per half of a key tile
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps; // + producer warp + MMA warp
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kBM = 128;                          // queries per tile
 constexpr uint32_t kTmemCols = 512;
+
+// Per-variant configuration.
+template <bool kMla>
+struct Cfg;
+
+// MLA: the Qa operand (128 x 224 bf16) sits in shared memory (SS MMAs for the
+// scores): O (192) + two 128-key S buffers (256) + Qa (112) would exceed the
+// 512 TMEM columns, and 128-key score tiles matter more than the A source
+// (a K = 16 tcgen05.mma takes at least ~93 cycles, so narrower N loses).
+template <>
+struct Cfg<true> {
+  static constexpr int kBN = 128;                              // keys per tile
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kBlkRows = 128 * 128;              // one 128B-swizzled block of a key tile
+  static constexpr uint32_t kStage = 3 * kBlkRows + 128 * 64;  // [c: 3 blocks | k_r: 128 x 64 B] = 57344
+  static constexpr uint32_t kQaBytes = kStage;                 // Qa tile, same block structure
+  static constexpr int kOCols = kDc;
+  static constexpr uint32_t kTmemS0 = 256, kTmemS1 = 384;
+};
+
+// Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
+template <>
+struct Cfg<false> {
+  static constexpr int kBN = 128;
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kBlkRows = 128 * 128;
+  static constexpr uint32_t kStage = 4 * kBlkRows;            // [K: 2 blocks | V: 2 blocks] = 65536
+  static constexpr uint32_t kQaBytes = 0;
+  static constexpr int kOCols = kDh;
+  static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
+};
+
+constexpr uint32_t kBlk128 = 128 * 128;  // 128 rows x 128 B: prologue / epilogue operand blocks
 constexpr uint32_t kTmemO = 0;
-constexpr uint32_t kTmemS0 = 256;
-constexpr uint32_t kTmemS1 = 384;
-constexpr uint32_t kTmemOA = 256;
-constexpr uint32_t kTmemOut = 384;
+
+template <bool kMla>
+struct Layout {
+  static constexpr uint32_t kRingOff = Cfg<kMla>::kQaBytes;
+  static constexpr uint32_t kBarOff = kRingOff + Cfg<kMla>::kStages * Cfg<kMla>::kStage;
+  static constexpr uint32_t kRedOff = kBarOff + 512;
+  static constexpr uint32_t kUsed = kRedOff + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
+  static constexpr uint32_t kMaxPad = kBytes - kUsed;  // alignment slack the kernel checks for
+};
+static_assert(Layout<true>::kBytes <= 232448, "MLA shared memory");
+static_assert(Layout<false>::kBytes <= 232448, "dense shared memory");
+static_assert(Layout<true>::kMaxPad >= 512 && Layout<false>::kMaxPad >= 512, "alignment slack");
+// The MLA prologue parks q (2 blocks) and W_UK (3 blocks) in the first ring stages.
+static_assert(5 * kBlk128 <= 2 * Cfg<true>::kStage, "prologue operands fit in stages 0-1");
+static_assert(2 * kBlk128 <= Cfg<true>::kStage && kBlk128 <= Cfg<true>::kStage, "W_UV blocks fit");
 
 enum Bar {
   B_PRO = 0, B_QABS, B_QA,
-  B_KVF0, B_KVF1, B_KVF2,
-  B_KVE0, B_KVE1, B_KVE2,
-  B_SF0, B_SF1,
+  B_KVF0,                   // kStages "full" barriers
+  B_KVE0 = B_KVF0 + 8,      // kStages "empty" barriers
+  B_SF0 = B_KVE0 + 8, B_SF1,
   B_PF0, B_PF1,
   B_PV, B_OA, B_OUT, B_DRAIN,
-  B_COUNT
+  B_MX0,                    // 8 barriers: (TMEM lane quadrant, tile parity)
+  B_COUNT = B_MX0 + 8
 };
+static_assert(B_COUNT * 8 + 8 <= 512, "barrier area");
 
 struct ChunkMaps {
   CUtensorMap q;    // [B, Nq, H, 128] box (64, 1, 128, 1), 128B swizzle
   CUtensorMap wuk;  // [H*128, 192]    box (64, 128), 128B swizzle
   CUtensorMap wuv;  // [H*128, 192]    box (64, 128), 128B swizzle
-  CUtensorMap c;    // [B, n_kv, 224]  box (64, 128, 1), 128B swizzle (content latent)
-  CUtensorMap kr;   // [B, n_kv, 224]  box (32, 128, 1), 64B swizzle (rope key, x = 192)
+  CUtensorMap c;    // [B, n_kv, 224]  box (64, 96, 1), 128B swizzle (content latent)
+  CUtensorMap kr;   // [B, n_kv, 224]  box (32, 96, 1), 64B swizzle (rope key, x = 192)
 };
 
 struct DenseMaps {
-  CUtensorMap q;  // [B, Nq, H, 128]
-  CUtensorMap k;  // [B, Nk, H, 128]
+  CUtensorMap k;  // [B, Nk, H, 128] box (64, 1, 128, 1)
   CUtensorMap v;  // [B, Nk, H, 128]
 };
 
 struct AttnParams {
+  const uint16_t* q;       // dense: queries are read directly into tensor memory
   const uint16_t* q_rope;  // MLA only
   uint16_t* out;
   int* status;
@@ -112,7 +163,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, ok);
 }
 
-// Write 8 packed bf16x2 words (16 B chunks) of row r into a 128B-swizzled block.
+// Write one 16-byte chunk of row r into a 128B- / 64B-swizzled block (shared memory).
 __device__ __forceinline__ void st_sw128_chunk(uint8_t* blk, int r, int chunk, uint4 v) {
   *reinterpret_cast<uint4*>(blk + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
 }
@@ -120,70 +171,122 @@ __device__ __forceinline__ void st_sw64_chunk(uint8_t* blk, int r, int chunk, ui
   *reinterpret_cast<uint4*>(blk + r * 64 + ((chunk ^ ((r >> 1) & 3)) << 4)) = v;
 }
 
-// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi, float scale) {
+  return pack_bf16x2(__uint_as_float(lo) * scale, __uint_as_float(hi) * scale);
+}
+__device__ __forceinline__ uint4 pack8(const uint32_t* v, float scale) {
+  return make_uint4(pack2(v[0], v[1], scale), pack2(v[2], v[3], scale), pack2(v[4], v[5], scale),
+                    pack2(v[6], v[7], scale));
+}
+
+// Softmax roles: thread (half, quadrant qd, lane) owns query row r = 32 qd + lane,
+// key columns [kBN/2 half, kBN/2 (half + 1)) of every S tile and output columns
+// [half kOCols/2, (half + 1) kOCols/2).  The two halves of a row agree on the row
+// maximum through `red` (shared memory, double-buffered by tile parity) and the
+// barrier B_MX0 + 2 qd + parity (64 arrivals: the two warps of the quadrant).
+struct SoftmaxThread {
+  uint32_t t_row;  // TMEM address of lane r, column 0
+  int half, qd, r;
+  float* red;      // [2 parity][2 half][128 rows]
+};
+
+// Exchange a per-row value with the other half; returns the partner's value.
+__device__ __forceinline__ bool exchange(const SoftmaxThread& t, uint32_t bars, int seq, float mine,
+                                         float& theirs, const WaitCtl& ctl) {
+  const int par = seq & 1;
+  t.red[(par * 2 + t.half) * 128 + t.r] = mine;
+  tc_fence_before();
+  mbar_arrive(bar_addr(bars, B_MX0 + 2 * t.qd + par));
+  if (!warp_wait(bar_addr(bars, B_MX0 + 2 * t.qd + par), (seq >> 1) & 1, ctl)) return false;
+  tc_fence_after();
+  theirs = t.red[(par * 2 + (t.half ^ 1)) * 128 + t.r];
+  return true;
+}
+
 // Softmax step for key tile j.  Returns false on abort.
-// ---------------------------------------------------------------------------
-template <int kOCols>
-__device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, uint32_t t_row,
+template <bool kMla>
+__device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const SoftmaxThread& t,
                                              const AttnParams& p, const WaitCtl& ctl,
-                                             float& m_run, float& l_run) {
+                                             float& m_run, float& l_part) {
+  using C = Cfg<kMla>;
+  constexpr int kW = C::kBN / 2;  // score columns per thread (48 or 64)
   const int sb = j & 1;
   if (!warp_wait(bar_addr(bars, B_SF0 + sb), (j >> 1) & 1, ctl)) return false;
   tc_fence_after();
-  const uint32_t scol = sb ? kTmemS1 : kTmemS0;
-  float s[kBN];
+  const uint32_t sbase = sb ? C::kTmemS1 : C::kTmemS0;
+  float s[kW];
   {
-    uint32_t r[32];
+    uint32_t ra[32], rb[kW - 32];
+    tmem_ld32(t.t_row + sbase + kW * t.half, ra);
+    if constexpr (kW - 32 == 16) tmem_ld16(t.t_row + sbase + kW * t.half + 32, rb);
+    else tmem_ld32(t.t_row + sbase + kW * t.half + 32, rb);
+    tmem_ld_wait();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      tmem_ld32(t_row + scol + 32 * c, r);
-      tmem_ld_wait();
+    for (int e = 0; e < 32; ++e) s[e] = __uint_as_float(ra[e]);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
-    }
+    for (int e = 0; e < kW - 32; ++e) s[32 + e] = __uint_as_float(rb[e]);
   }
-  const int64_t kv0 = (int64_t)j * kBN;
-  if (kv0 + kBN > p.n_kv) {
-    const int valid = (int)(p.n_kv - kv0);
+  const int64_t kv0 = (int64_t)j * C::kBN + kW * t.half;
+  if (kv0 + kW > p.n_kv) {
+    const int64_t valid = p.n_kv - kv0;  // may be <= 0: the whole half is padding
 #pragma unroll
-    for (int c = 0; c < kBN; ++c)
+    for (int c = 0; c < kW; ++c)
       if (c >= valid) s[c] = -INFINITY;
   }
-  float mx = s[0];
+  float mx[8];
 #pragma unroll
-  for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
-  const float m_tile = mx * p.scale_log2;
+  for (int c = 0; c < 8; ++c) mx[c] = s[c];
+#pragma unroll
+  for (int c = 8; c < kW; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+  mx[0] = fmaxf(mx[0], mx[4]); mx[1] = fmaxf(mx[1], mx[5]);
+  mx[2] = fmaxf(mx[2], mx[6]); mx[3] = fmaxf(mx[3], mx[7]);
+  mx[0] = fmaxf(mx[0], mx[2]); mx[1] = fmaxf(mx[1], mx[3]);
+  const float lmax = fmaxf(mx[0], mx[1]);
+  // The partner's columns of S are read before either half writes P over them.
+  float omax;
+  if (!exchange(t, bars, j, lmax, omax, ctl)) return false;
+  const float m_tile = fmaxf(lmax, omax) * p.scale_log2;
   const bool need = m_tile > m_run + 8.0f;
   const float m_new = need ? m_tile : m_run;
   const float alpha = fast_exp2(m_run - m_new);
-  float sum = 0.0f;
+  float sum[8];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t pk[16];
+  for (int c = 0; c < 8; ++c) sum[c] = 0.0f;
+  uint32_t pk[kW / 2];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float p0 = fast_exp2(fmaf(s[32 * c + 2 * e], p.scale_log2, -m_new));
-      const float p1 = fast_exp2(fmaf(s[32 * c + 2 * e + 1], p.scale_log2, -m_new));
-      sum += p0 + p1;
-      pk[e] = pack_bf16x2(p0, p1);
-    }
-    tmem_st16(t_row + scol + 16 * c, pk);
+  for (int e = 0; e < kW / 2; ++e) {
+    const float p0 = fast_exp2(fmaf(s[2 * e], p.scale_log2, -m_new));
+    const float p1 = fast_exp2(fmaf(s[2 * e + 1], p.scale_log2, -m_new));
+    sum[(2 * e) & 7] += p0;
+    sum[(2 * e + 1) & 7] += p1;
+    pk[e] = pack_bf16x2(p0, p1);
   }
-  l_run = l_run * alpha + sum;
-  if (j > 0) {
-    // O may only be touched once the previous P.C product has landed.
+  // P (bf16 pairs) over the first kBN/2 cells of the S buffer: this half's kW/2 cells.
+  const uint32_t pcol = t.t_row + sbase + (kW / 2) * t.half;
+  if constexpr (kW / 2 == 24) {
+    tmem_st16(pcol, pk);
+    tmem_st8(pcol + 16, pk + 16);
+  } else {
+    tmem_st32(pcol, pk);
+  }
+  sum[0] += sum[4]; sum[1] += sum[5]; sum[2] += sum[6]; sum[3] += sum[7];
+  sum[0] += sum[2]; sum[1] += sum[3];
+  l_part = l_part * alpha + (sum[0] + sum[1]);
+  if (j > 0 && __any_sync(0xffffffffu, need)) {
+    // O may only be rescaled once the previous P.C product has landed.  The PV
+    // barrier cannot run ahead of PV(j-1) (PV(j) needs this tile's P), so its
+    // parity identifies that phase even when earlier phases were not waited on.
     if (!warp_wait(bar_addr(bars, B_PV), (j - 1) & 1, ctl)) return false;
-    if (__any_sync(0xffffffffu, need)) {
-      tc_fence_after();
-      uint32_t r[32];
+    tc_fence_after();
+    uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < kOCols / 32; ++c) {
-        tmem_ld32(t_row + kTmemO + 32 * c, r);
-        tmem_ld_wait();
+    for (int c = 0; c < C::kOCols / 64; ++c) {
+      const uint32_t col = kTmemO + t.half * (C::kOCols / 2) + 32 * c;
+      tmem_ld32(t.t_row + col, r);
+      tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-        tmem_st32(t_row + kTmemO + 32 * c, r);
-      }
+      for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+      tmem_st32(t.t_row + col, r);
     }
   }
   tmem_st_wait();
@@ -194,19 +297,30 @@ __device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, uint32_t t_ro
 }
 
 // ---------------------------------------------------------------------------
-// MLA chunk attention
+// The attention kernel.  kMla: latent chunk attention (absorbed W_UK, [c ; k_r]
+// tiles, W_UV epilogue); otherwise the dense per-head baseline (d = 128).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1)
-    k_chunk_attn(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
-                 const __grid_constant__ RopeTable tab) {
+template <bool kMla, class Maps>
+__device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p, const RopeTable* tab) {
+  using C = Cfg<kMla>;
+  using L = Layout<kMla>;
+  constexpr int kBN = C::kBN;
+  constexpr int kStages = C::kStages;
+  constexpr uint32_t kStage = C::kStage;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t s_base = smem_u32(smem);
-  const uint32_t qa = s_base;                 // Qa tile: 3 x 128B-swizzled blocks + rope block
-  const uint32_t st0 = s_base + kMlaStage;    // stage s at st0 + s * kMlaStage
-  const uint32_t bars = s_base + kSmemBarOff;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSmemBarOff + 8 * B_COUNT);
+  const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
+  const uint32_t pad = (uint32_t)(((raw + 1023) & ~uintptr_t(1023)) - raw);
+  if (pad > L::kMaxPad) {  // uniform across the CTA: nothing has started yet
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kDevSmemMisaligned);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t qa = smem_u32(smem);    // MLA: Qa tile (3 SW128 blocks + SW64 rope block)
+  const uint32_t st0 = qa + L::kRingOff; // ring stage s at st0 + s * kStage
+  const uint32_t bars = qa + L::kBarOff;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -218,19 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_addr(bars, B_PRO), 1);
     mbar_init(bar_addr(bars, B_QABS), 1);
-    mbar_init(bar_addr(bars, B_QA), 128);
+    mbar_init(bar_addr(bars, B_QA), kSoftmaxThreads);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar_addr(bars, B_KVF0 + s), 1);
       mbar_init(bar_addr(bars, B_KVE0 + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_addr(bars, B_SF0 + s), 1);
-      mbar_init(bar_addr(bars, B_PF0 + s), 128);
+      mbar_init(bar_addr(bars, B_PF0 + s), kSoftmaxThreads);
     }
     mbar_init(bar_addr(bars, B_PV), 1);
-    mbar_init(bar_addr(bars, B_OA), 128);
+    mbar_init(bar_addr(bars, B_OA), kSoftmaxThreads);
     mbar_init(bar_addr(bars, B_OUT), 1);
     mbar_init(bar_addr(bars, B_DRAIN), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar_addr(bars, B_MX0 + i), 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -247,48 +362,67 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------- producer -------------------------------
-      tma_prefetch_desc(&maps.q);
-      tma_prefetch_desc(&maps.wuk);
-      tma_prefetch_desc(&maps.wuv);
-      tma_prefetch_desc(&maps.c);
-      tma_prefetch_desc(&maps.kr);
-      const uint32_t st1 = st0 + kMlaStage;
-      mbar_arrive_expect_tx(bar_addr(bars, B_PRO), 2 * kBlk + 3 * kBlk);
-      tma_load_4d(st0, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
-      tma_load_4d(st0 + kBlk, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
-      tma_load_2d(st1, &maps.wuk, bar_addr(bars, B_PRO), 0, h * kDh);
-      tma_load_2d(st1 + kBlk, &maps.wuk, bar_addr(bars, B_PRO), 64, h * kDh);
-      tma_load_2d(st1 + 2 * kBlk, &maps.wuk, bar_addr(bars, B_PRO), 128, h * kDh);
-      int last_use[kStages] = {-1, -1, -1};
+      int last_use[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last_use[s] = -1;
       bool ok = true;
-      for (int i = 0; i <= n_tiles; ++i) {
+      if constexpr (kMla) {
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.wuk);
+        tma_prefetch_desc(&maps.wuv);
+        tma_prefetch_desc(&maps.c);
+        tma_prefetch_desc(&maps.kr);
+        // Prologue operands borrow ring stages 0-1: q tile (2 blocks) then W_UK_h (3 blocks).
+        mbar_arrive_expect_tx(bar_addr(bars, B_PRO), 5 * kBlk128);
+        tma_load_4d(st0, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
+        tma_load_4d(st0 + kBlk128, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
+        tma_load_2d(st0 + 2 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 0, h * kDh);
+        tma_load_2d(st0 + 3 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 64, h * kDh);
+        tma_load_2d(st0 + 4 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 128, h * kDh);
+      } else {
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+      }
+      // MLA: n_tiles key tiles, then W_UV_h blocks {0,1} and {2} as two more ring items.
+      const int n_items = kMla ? n_tiles + 2 : n_tiles;
+      for (int i = 0; i < n_items; ++i) {
         const int st = i % kStages, use = i / kStages;
-        const uint32_t sa = st0 + st * kMlaStage;
+        const uint32_t sa = st0 + st * kStage;
         if (use == 0) {
-          if (st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
+          if (kMla && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
         } else {
           ok = mbar_wait(bar_addr(bars, B_KVE0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer);
         }
         if (!ok) break;
         const uint32_t fb = bar_addr(bars, B_KVF0 + st);
-        if (i < n_tiles) {
-          const int kv0 = i * kBN;
-          mbar_arrive_expect_tx(fb, kMlaStage);
-          tma_load_3d(sa, &maps.c, fb, 0, kv0, b);
-          tma_load_3d(sa + kBlk, &maps.c, fb, 64, kv0, b);
-          tma_load_3d(sa + 2 * kBlk, &maps.c, fb, 128, kv0, b);
-          tma_load_3d(sa + 3 * kBlk, &maps.kr, fb, kDc, kv0, b);
+        const int kv0 = i * kBN;
+        if constexpr (kMla) {
+          if (i < n_tiles) {
+            mbar_arrive_expect_tx(fb, kStage);
+            tma_load_3d(sa, &maps.c, fb, 0, kv0, b);
+            tma_load_3d(sa + C::kBlkRows, &maps.c, fb, 64, kv0, b);
+            tma_load_3d(sa + 2 * C::kBlkRows, &maps.c, fb, 128, kv0, b);
+            tma_load_3d(sa + 3 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
+          } else if (i == n_tiles) {
+            mbar_arrive_expect_tx(fb, 2 * kBlk128);
+            tma_load_2d(sa, &maps.wuv, fb, 0, h * kDh);
+            tma_load_2d(sa + kBlk128, &maps.wuv, fb, 64, h * kDh);
+          } else {
+            mbar_arrive_expect_tx(fb, kBlk128);
+            tma_load_2d(sa, &maps.wuv, fb, 128, h * kDh);
+          }
         } else {
-          mbar_arrive_expect_tx(fb, 3 * kBlk);
-          tma_load_2d(sa, &maps.wuv, fb, 0, h * kDh);
-          tma_load_2d(sa + kBlk, &maps.wuv, fb, 64, h * kDh);
-          tma_load_2d(sa + 2 * kBlk, &maps.wuv, fb, 128, h * kDh);
+          mbar_arrive_expect_tx(fb, kStage);
+          tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
+          tma_load_4d(sa + C::kBlkRows, &maps.k, fb, 64, h, kv0, b);
+          tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, h, kv0, b);
+          tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, h, kv0, b);
         }
         last_use[st] = use;
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits.
-        drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
+        if (kMla) drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
         for (int s = 0; s < kStages; ++s)
           if (last_use[s] >= 0)
             drain_wait(bar_addr(bars, B_KVF0 + s), last_use[s] & 1, p.wait_limit_ns, p.status);
@@ -297,33 +431,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // --------------------------------- MMA ----------------------------------
-      constexpr uint32_t kIdQabs = idesc_bf16_f32(128, 192, false, true);
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdPv = idesc_bf16_f32(128, 192, false, true);
-      constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t st1 = st0 + kMlaStage;
-      bool ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
-      if (ok) {
-        tc_fence_after();
-        // q_abs = q_h . W_UK_h  (M 128, N 192, K 128); q K-major, W_UK MN-major.
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, kBN, false, false);
+      constexpr uint32_t kIdPv = idesc_bf16_f32(128, C::kOCols, false, true);
+      bool ok = true;
+      if constexpr (kMla) {
+        ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
+        if (ok) {
+          constexpr uint32_t kIdQabs = idesc_bf16_f32(128, kDc, false, true);
+          tc_fence_after();
+          // q_abs = q_h . W_UK_h (M 128, N 192, K 128): q K-major, W_UK MN-major.
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk + (k & 3) * 32, 16, 1024, kSw128);
-          const uint64_t bd = smem_desc(st1 + k * 2048, kBlk, 1024, kSw128);
-          umma_ss(tmem + kTmemO, a, bd, kIdQabs, k > 0);
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
+            const uint64_t bd = smem_desc(st0 + 2 * kBlk128 + k * 2048, kBlk128, 1024, kSw128);
+            umma_ss(tmem + kTmemO, a, bd, kIdQabs, k > 0);
+          }
+          umma_commit(bar_addr(bars, B_QABS));
         }
-        umma_commit(bar_addr(bars, B_QABS));
-        ok = mbar_wait(bar_addr(bars, B_QA), 0, ctl, kDevTimeoutMma);
       }
+      if (ok) ok = mbar_wait(bar_addr(bars, B_QA), 0, ctl, kDevTimeoutMma);
       auto issue_pv = [&](int jj) -> bool {
         if (!mbar_wait(bar_addr(bars, B_PF0 + (jj & 1)), (jj >> 1) & 1, ctl, kDevTimeoutMma))
           return false;
         tc_fence_after();
-        const uint32_t sa = st0 + (jj % kStages) * kMlaStage;
-        const uint32_t a_t = tmem + ((jj & 1) ? kTmemS1 : kTmemS0);
+        // V operand: the latent c blocks (MLA) or the V blocks (dense), MN-major.
+        const uint32_t sv = st0 + (jj % kStages) * kStage + (kMla ? 0u : 2 * C::kBlkRows);
+        const uint32_t a_t = tmem + ((jj & 1) ? C::kTmemS1 : C::kTmemS0);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(sa + k * 2048, kBlk, 1024, kSw128);
+        for (int k = 0; k < kBN / 16; ++k) {
+          const uint64_t bd = smem_desc(sv + k * 2048, C::kBlkRows, 1024, kSw128);
           umma_ts(tmem + kTmemO, a_t + k * 8, bd, kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(bar_addr(bars, B_PV));
@@ -335,40 +471,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(bar_addr(bars, B_KVF0 + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = st0 + st * kMlaStage;
-        const uint32_t d = tmem + ((j & 1) ? kTmemS1 : kTmemS0);
+        const uint32_t sa = st0 + st * kStage;
+        const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+        if constexpr (kMla) {
+          // S = Qa . [c ; k_r]^T (K = 224): 12 steps over the 128B-swizzled content
+          // blocks, 2 over the 64B-swizzled rope block; Qa and the key tile share offsets.
 #pragma unroll
-        for (int k = 0; k < 14; ++k) {
-          uint64_t a, bd;
-          if (k < 12) {
-            const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
-            a = smem_desc(qa + off, 16, 1024, kSw128);
-            bd = smem_desc(sa + off, 16, 1024, kSw128);
-          } else {
-            const uint32_t off = 3 * kBlk + (k - 12) * 32;
-            a = smem_desc(qa + off, 16, 512, kSw64);
-            bd = smem_desc(sa + off, 16, 512, kSw64);
+          for (int k = 0; k < 14; ++k) {
+            const uint32_t off = k < 12 ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : 3 * C::kBlkRows + (k - 12) * 32;
+            const uint32_t sbo = k < 12 ? 1024 : 512;
+            const uint32_t lay = k < 12 ? kSw128 : kSw64;
+            umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
           }
-          umma_ss(d, a, bd, kIdS, k > 0);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t bd = smem_desc(sa + (k >> 2) * C::kBlkRows + (k & 3) * 32, 16, 1024, kSw128);
+            umma_ts(d, tmem + C::kTmemQ + k * 8, bd, kIdS, k > 0);
+          }
         }
         umma_commit(bar_addr(bars, B_SF0 + (j & 1)));
         if (j >= 1) ok = issue_pv(j - 1);
       }
       if (ok) ok = issue_pv(n_tiles - 1);
-      if (ok) {
-        const int st = n_tiles % kStages;
-        ok = mbar_wait(bar_addr(bars, B_KVF0 + st), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
-             mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
+      if constexpr (kMla) {
         if (ok) {
-          tc_fence_after();
-          const uint32_t sa = st0 + st * kMlaStage;
-          // out = O_lat/l . W_UV_h^T  (M 128, N 128, K 192); A from TMEM, W_UV K-major.
+          constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
+          const int s01 = n_tiles % kStages, s2 = (n_tiles + 1) % kStages;
+          ok = mbar_wait(bar_addr(bars, B_KVF0 + s01), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
+               mbar_wait(bar_addr(bars, B_KVF0 + s2), ((n_tiles + 1) / kStages) & 1, ctl, kDevTimeoutMma) &&
+               mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t wb[3] = {st0 + s01 * kStage, st0 + s01 * kStage + kBlk128, st0 + s2 * kStage};
+            // out = O_lat/l . W_UV_h^T (M 128, N 128, K 192): A from TMEM, W_UV K-major.
 #pragma unroll
-          for (int k = 0; k < 12; ++k) {
-            const uint64_t bd = smem_desc(sa + (k >> 2) * kBlk + (k & 3) * 32, 16, 1024, kSw128);
-            umma_ts(tmem + kTmemOut, tmem + kTmemOA + k * 8, bd, kIdOut, k > 0);
+            for (int k = 0; k < 12; ++k) {
+              const uint64_t bd = smem_desc(wb[k >> 2] + (k & 3) * 32, 16, 1024, kSw128);
+              umma_ts(tmem + C::kTmemS1, tmem + C::kTmemS0 + k * 8, bd, kIdOut, k > 0);
+            }
+            umma_commit(bar_addr(bars, B_OUT));
           }
-          umma_commit(bar_addr(bars, B_OUT));
         }
       }
       if (!ok) {
@@ -378,111 +521,141 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------- softmax ---------------------------------
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;
-    const uint32_t t_row = tmem + ((uint32_t)(qd * 32) << 16);
-    const int qi = q0 + r;
-    bool ok = warp_wait(bar_addr(bars, B_QABS), 0, ctl);
-    if (ok) {
-      tc_fence_after();
-      uint8_t* qa_p = smem;
+    SoftmaxThread t;
+    t.qd = warp & 3;
+    t.half = (warp - 2) >> 2;
+    t.r = t.qd * 32 + lane;
+    t.t_row = tmem + ((uint32_t)(t.qd * 32) << 16);
+    t.red = red;
+    const int qi = q0 + t.r;
+    bool ok = true;
+    if constexpr (kMla) {
+      ok = warp_wait(bar_addr(bars, B_QABS), 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        // q_abs (fp32, TMEM) -> bf16 Qa tile in shared memory; this half: columns [96 half, +96).
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          const int col = 96 * t.half + 32 * c;
+          tmem_ld32(t.t_row + kTmemO + col, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            st_sw128_chunk(smem + (col >> 6) * C::kBlkRows, t.r, ((col & 63) >> 3) + q4, pack8(v + 8 * q4, 1.0f));
+        }
+        if (t.half == 0) {
+          // Rope part of the query, rotated with the query's own (t, row, col).
+          float qr[kDr];
+#pragma unroll
+          for (int e = 0; e < kDr; ++e) qr[e] = 0.0f;
+          if (qi < p.n_q) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                p.q_rope + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDr);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 u = __ldg(src + c);
+              qr[8 * c + 0] = bf16lo_to_f32(u.x); qr[8 * c + 1] = bf16hi_to_f32(u.x);
+              qr[8 * c + 2] = bf16lo_to_f32(u.y); qr[8 * c + 3] = bf16hi_to_f32(u.y);
+              qr[8 * c + 4] = bf16lo_to_f32(u.z); qr[8 * c + 5] = bf16hi_to_f32(u.z);
+              qr[8 * c + 6] = bf16lo_to_f32(u.w); qr[8 * c + 7] = bf16hi_to_f32(u.w);
+            }
+            const int per_frame = p.grid_h * p.grid_w;
+            const int f = qi / per_frame;
+            const int rem = qi - f * per_frame;
+            const int row = rem / p.grid_w;
+            const int col = rem - row * p.grid_w;
+#pragma unroll
+            for (int pr = 0; pr < kDr / 2; ++pr) {
+              float2 cs;
+              if (pr < kPairsT) cs = tab->t[f][pr];
+              else if (pr < kPairsT + kPairsH) cs = tab->h[row][pr - kPairsT];
+              else cs = tab->w[col][pr - kPairsT - kPairsH];
+              const float a = qr[2 * pr], bb = qr[2 * pr + 1];
+              qr[2 * pr] = a * cs.x - bb * cs.y;
+              qr[2 * pr + 1] = a * cs.y + bb * cs.x;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 w;
+            w.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
+            w.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
+            w.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
+            w.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
+            st_sw64_chunk(smem + 3 * C::kBlkRows, t.r, c, w);
+          }
+        }
+        fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
+      }
+    } else {
+      // Dense queries straight from global memory into the Q cells (bf16 pairs).
       uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < 6; ++c) {
-        tmem_ld32(t_row + kTmemO + 32 * c, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]), __uint_as_float(v[8 * q4 + 1]));
-          w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3]));
-          w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5]));
-          w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
-          st_sw128_chunk(qa_p + (c >> 1) * kBlk, r, (c & 1) * 4 + q4, w);
-        }
-      }
-      // Rope part of the query, rotated with the query's own (t, row, col).
-      float qr[kDr];
-#pragma unroll
-      for (int e = 0; e < kDr; ++e) qr[e] = 0.0f;
+      for (int e = 0; e < 32; ++e) v[e] = 0u;
       if (qi < p.n_q) {
         const uint4* src = reinterpret_cast<const uint4*>(
-            p.q_rope + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDr);
+            p.q + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh + 64 * t.half);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           const uint4 u = __ldg(src + c);
-          qr[8 * c + 0] = bf16lo_to_f32(u.x); qr[8 * c + 1] = bf16hi_to_f32(u.x);
-          qr[8 * c + 2] = bf16lo_to_f32(u.y); qr[8 * c + 3] = bf16hi_to_f32(u.y);
-          qr[8 * c + 4] = bf16lo_to_f32(u.z); qr[8 * c + 5] = bf16hi_to_f32(u.z);
-          qr[8 * c + 6] = bf16lo_to_f32(u.w); qr[8 * c + 7] = bf16hi_to_f32(u.w);
-        }
-        const int per_frame = p.grid_h * p.grid_w;
-        const int f = qi / per_frame;
-        const int rem = qi - f * per_frame;
-        const int row = rem / p.grid_w;
-        const int col = rem - row * p.grid_w;
-#pragma unroll
-        for (int pr = 0; pr < kDr / 2; ++pr) {
-          float2 cs;
-          if (pr < kPairsT) cs = tab.t[f][pr];
-          else if (pr < kPairsT + kPairsH) cs = tab.h[row][pr - kPairsT];
-          else cs = tab.w[col][pr - kPairsT - kPairsH];
-          const float a = qr[2 * pr], bb = qr[2 * pr + 1];
-          qr[2 * pr] = a * cs.x - bb * cs.y;
-          qr[2 * pr + 1] = a * cs.y + bb * cs.x;
+          v[4 * c + 0] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
         }
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 w;
-        w.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
-        w.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
-        w.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
-        w.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
-        st_sw64_chunk(qa_p + 3 * kBlk, r, c, w);
-      }
-      fence_proxy_async_smem();
+      tmem_st32(t.t_row + C::kTmemQ + 32 * t.half, v);
+    }
+    if (ok) {
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_addr(bars, B_QA));
     }
-    float m_run = -INFINITY, l_run = 0.0f;
-    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kDc>(j, bars, t_row, p, ctl, m_run, l_run);
+    float m_run = -INFINITY, l_part = 0.0f;
+    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kMla>(j, bars, t, p, ctl, m_run, l_part);
+    float l_other = 0.0f;
+    if (ok) ok = exchange(t, bars, n_tiles, l_part, l_other, ctl);
     if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l_run;
+      const float inv_l = 1.0f / (l_part + l_other);
+      uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
       uint32_t v[32];
+      if constexpr (kMla) {
+        // Normalised O_lat -> bf16 A operand of the W_UV MMA (this half: latent [96 half, +96)).
 #pragma unroll
-      for (int c = 0; c < 6; ++c) {
-        tmem_ld32(t_row + kTmemO + 32 * c, v);
-        tmem_ld_wait();
-        uint32_t pk[16];
+        for (int c = 0; c < 3; ++c) {
+          tmem_ld32(t.t_row + kTmemO + 96 * t.half + 32 * c, v);
+          tmem_ld_wait();
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv_l, __uint_as_float(v[2 * e + 1]) * inv_l);
-        tmem_st16(t_row + kTmemOA + 16 * c, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_addr(bars, B_OA));
-      ok = warp_wait(bar_addr(bars, B_OUT), 0, ctl);
-      if (ok) {
-        tc_fence_after();
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh);
+          for (int e = 0; e < 16; ++e) pk[e] = pack2(v[2 * e], v[2 * e + 1], inv_l);
+          tmem_st16(t.t_row + C::kTmemS0 + 48 * t.half + 16 * c, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_addr(bars, B_OA));
+        ok = warp_wait(bar_addr(bars, B_OUT), 0, ctl);
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(t_row + kTmemOut + 32 * c, v);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(t.t_row + C::kTmemS1 + 64 * t.half + 32 * c, v);
+            tmem_ld_wait();
+            if (qi < p.n_q) {
+              uint4* dst = reinterpret_cast<uint4*>(out_row + 64 * t.half + 32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) dst[q4] = pack8(v + 8 * q4, 1.0f);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(t.t_row + kTmemO + 64 * t.half + 32 * c, v);
           tmem_ld_wait();
           if (qi < p.n_q) {
+            uint4* dst = reinterpret_cast<uint4*>(out_row + 64 * t.half + 32 * c);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]), __uint_as_float(v[8 * q4 + 1]));
-              w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3]));
-              w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5]));
-              w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
-              dst[4 * c + q4] = w;
-            }
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = pack8(v + 8 * q4, inv_l);
           }
         }
       }
@@ -498,165 +671,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// Dense per-head attention (d = 128), same skeleton without the projections
-// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1)
+    k_chunk_attn(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
+                 const __grid_constant__ RopeTable tab) {
+  attn_body<true>(maps, p, &tab);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_dense_attn(const __grid_constant__ DenseMaps maps, const __grid_constant__ AttnParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t s_base = smem_u32(smem);
-  const uint32_t qs = s_base;                 // Q tile: 2 x 128B-swizzled blocks
-  const uint32_t st0 = s_base + 2 * kBlk;     // stage s at st0 + s * kDenseStage
-  const uint32_t bars = s_base + kSmemBarOff;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kSmemBarOff + 8 * B_COUNT);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x % p.heads;
-  const int q0 = (blockIdx.x / p.heads) * kBM;
-  const int b = blockIdx.y;
-  const int n_tiles = p.n_kv_tiles;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar_addr(bars, B_PRO), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_addr(bars, B_KVF0 + s), 1);
-      mbar_init(bar_addr(bars, B_KVE0 + s), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_addr(bars, B_SF0 + s), 1);
-      mbar_init(bar_addr(bars, B_PF0 + s), 128);
-    }
-    mbar_init(bar_addr(bars, B_PV), 1);
-    mbar_init(bar_addr(bars, B_DRAIN), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
-
-  if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&maps.q);
-      tma_prefetch_desc(&maps.k);
-      tma_prefetch_desc(&maps.v);
-      mbar_arrive_expect_tx(bar_addr(bars, B_PRO), 2 * kBlk);
-      tma_load_4d(qs, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
-      tma_load_4d(qs + kBlk, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
-      int last_use[kStages] = {-1, -1, -1};
-      bool ok = true;
-      for (int i = 0; i < n_tiles; ++i) {
-        const int st = i % kStages, use = i / kStages;
-        const uint32_t sa = st0 + st * kDenseStage;
-        if (use > 0) ok = mbar_wait(bar_addr(bars, B_KVE0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer);
-        if (!ok) break;
-        const uint32_t fb = bar_addr(bars, B_KVF0 + st);
-        const int kv0 = i * kBN;
-        mbar_arrive_expect_tx(fb, kDenseStage);
-        tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
-        tma_load_4d(sa + kBlk, &maps.k, fb, 64, h, kv0, b);
-        tma_load_4d(sa + 2 * kBlk, &maps.v, fb, 0, h, kv0, b);
-        tma_load_4d(sa + 3 * kBlk, &maps.v, fb, 64, h, kv0, b);
-        last_use[st] = use;
-      }
-      if (!ok) {
-        drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
-        for (int s = 0; s < kStages; ++s)
-          if (last_use[s] >= 0)
-            drain_wait(bar_addr(bars, B_KVF0 + s), last_use[s] & 1, p.wait_limit_ns, p.status);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdPv = idesc_bf16_f32(128, 128, false, true);
-      bool ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(bar_addr(bars, B_PF0 + (jj & 1)), (jj >> 1) & 1, ctl, kDevTimeoutMma))
-          return false;
-        tc_fence_after();
-        const uint32_t sv = st0 + (jj % kStages) * kDenseStage + 2 * kBlk;
-        const uint32_t a_t = tmem + ((jj & 1) ? kTmemS1 : kTmemS0);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(sv + k * 2048, kBlk, 1024, kSw128);
-          umma_ts(tmem + kTmemO, a_t + k * 8, bd, kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_addr(bars, B_PV));
-        umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
-        return true;
-      };
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % kStages;
-        ok = mbar_wait(bar_addr(bars, B_KVF0 + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t sa = st0 + st * kDenseStage;
-        const uint32_t d = tmem + ((j & 1) ? kTmemS1 : kTmemS0);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
-          umma_ss(d, smem_desc(qs + off, 16, 1024, kSw128), smem_desc(sa + off, 16, 1024, kSw128),
-                  kIdS, k > 0);
-        }
-        umma_commit(bar_addr(bars, B_SF0 + (j & 1)));
-        if (j >= 1) ok = issue_pv(j - 1);
-      }
-      if (ok) ok = issue_pv(n_tiles - 1);
-      if (!ok) {
-        umma_commit(bar_addr(bars, B_DRAIN));
-        drain_wait(bar_addr(bars, B_DRAIN), 0, p.wait_limit_ns, p.status);
-      }
-    }
-  } else {
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;
-    const uint32_t t_row = tmem + ((uint32_t)(qd * 32) << 16);
-    const int qi = q0 + r;
-    float m_run = -INFINITY, l_run = 0.0f;
-    bool ok = true;
-    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kDh>(j, bars, t_row, p, ctl, m_run, l_run);
-    if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh);
-      uint32_t v[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(t_row + kTmemO + 32 * c, v);
-        tmem_ld_wait();
-        if (qi < p.n_q) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv_l, __uint_as_float(v[8 * q4 + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv_l, __uint_as_float(v[8 * q4 + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv_l, __uint_as_float(v[8 * q4 + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv_l, __uint_as_float(v[8 * q4 + 7]) * inv_l);
-            dst[4 * c + q4] = w;
-          }
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
+  attn_body<false>(maps, p, nullptr);
 }
 
 // ---------------------------------------------------------------------------
@@ -691,24 +714,25 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
-bool set_smem_attr(const void* fn, bool* done) {
+bool set_smem_attr(const void* fn, int bytes, bool* done) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
 }
 
-bool make_qmap(CUtensorMap* m, const uint16_t* q, int batch, int n_rows, int heads) {
+// [B, rows, H, 128] bf16, box of 128 rows x 64 elements of one head.
+bool make_head_map(CUtensorMap* m, const uint16_t* t, int batch, int64_t n_rows, int heads) {
   const cuuint64_t dims[4] = {(cuuint64_t)kDh, (cuuint64_t)heads, (cuuint64_t)n_rows, (cuuint64_t)batch};
   const cuuint64_t strides[3] = {(cuuint64_t)kDh * 2, (cuuint64_t)heads * kDh * 2,
                                  (cuuint64_t)n_rows * heads * kDh * 2};
   const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBM, 1};
-  return make_map(m, q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map(m, t, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -720,9 +744,9 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
                                    cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_chunk_attn, attr_done)) return cudaErrorInvalidValue;
+  if (!set_smem_attr((const void*)k_chunk_attn, Layout<true>::kBytes, attr_done)) return cudaErrorInvalidValue;
   ChunkMaps maps;
-  bool ok = make_qmap(&maps.q, q, batch, n_q, heads);
+  bool ok = make_head_map(&maps.q, q, batch, n_q, heads);
   {
     const cuuint64_t dims[2] = {(cuuint64_t)kDc, (cuuint64_t)heads * kDh};
     const cuuint64_t strides[1] = {(cuuint64_t)kDc * 2};
@@ -733,8 +757,8 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   {
     const cuuint64_t dims[3] = {(cuuint64_t)kDrow, (cuuint64_t)n_kv, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)kDrow * 2, (cuuint64_t)cap * kDrow * 2};
-    const cuuint32_t box_c[3] = {64, (cuuint32_t)kBN, 1};
-    const cuuint32_t box_r[3] = {32, (cuuint32_t)kBN, 1};
+    const cuuint32_t box_c[3] = {64, (cuuint32_t)Cfg<true>::kBN, 1};
+    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<true>::kBN, 1};
     ok = ok && make_map(&maps.c, cache, 3, dims, strides, box_c, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&maps.kr, cache, 3, dims, strides, box_r, CU_TENSOR_MAP_SWIZZLE_64B);
   }
@@ -743,6 +767,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
     return cudaErrorInvalidValue;
   }
   AttnParams p{};
+  p.q = q;
   p.q_rope = q_rope;
   p.out = out;
   p.status = status;
@@ -750,7 +775,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + kBN - 1) / kBN);
+  p.n_kv_tiles = (int)((n_kv + Cfg<true>::kBN - 1) / Cfg<true>::kBN);
   p.grid_h = grid_h;
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -758,7 +783,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_chunk_attn<<<grid, kThreads, kSmemBytes, stream>>>(maps, p, tab);
+  k_chunk_attn<<<grid, kThreads, Layout<true>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 
@@ -767,25 +792,25 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
                                    int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_dense_attn, attr_done)) return cudaErrorInvalidValue;
+  if (!set_smem_attr((const void*)k_dense_attn, Layout<false>::kBytes, attr_done)) return cudaErrorInvalidValue;
   DenseMaps maps;
-  bool ok = make_qmap(&maps.q, q, batch, n_q, heads) && make_qmap(&maps.k, k, batch, (int)n_kv, heads) &&
-            make_qmap(&maps.v, v, batch, (int)n_kv, heads);
+  bool ok = make_head_map(&maps.k, k, batch, n_kv, heads) && make_head_map(&maps.v, v, batch, n_kv, heads);
   if (!ok) {
     *encode_failed = true;
     return cudaErrorInvalidValue;
   }
   AttnParams p{};
+  p.q = q;
   p.out = out;
   p.status = status;
   p.wait_limit_ns = kWaitLimitNs;
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + kBN - 1) / kBN);
+  p.n_kv_tiles = (int)((n_kv + Cfg<false>::kBN - 1) / Cfg<false>::kBN);
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_dense_attn<<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+  k_dense_attn<<<grid, kThreads, Layout<false>::kBytes, stream>>>(maps, p);
   return cudaGetLastError();
 }
 
