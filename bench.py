@@ -9,8 +9,10 @@ queries, a 21-frame window = 32760 keys, 12 heads x 128, d_c = 192, d_r = 32):
     vmla_cache_append     the chunk's 4680 tokens -> [c ; RoPE3D(k_r)] rows of the window
     vmla_chunk_attention  4680 queries x 12 heads over the 32760 cached keys
 Inputs are seeded synthetic data (see the `workload` package) already resident in
-HBM when the timed region starts; L2 is flushed (256 MiB write) before every timed
-step.  `value` counts the absorbed-MLA tensor FLOPs of the attention,
+HBM when the timed region starts.  L2 is flushed before every timed step: a 256 MiB
+write evicts every cached line, then a 256 MiB read of a second buffer forces the
+write-back of those dirty lines, so the timed step starts from a cold, clean L2.
+`value` counts the absorbed-MLA tensor FLOPs of the attention,
 2*B*Nq*H*Nkv*(224+192), plus the append's 2*B*Nq*224*1536, per second.  The dense
 per-head baseline (3072 scalars/token) is timed on the same queries beside it.
 
@@ -65,7 +67,7 @@ def workload_desc(w) -> dict:
                      f"({w.cached_frames} cached + chunk), H={w.heads}x{w.d_head}, d_c={w.d_c}, d_r={w.d_r}"),
         "batch": w.batch, "n_q": w.n_q, "n_kv": w.n_kv, "heads": w.heads, "d_c": w.d_c, "d_r": w.d_r,
         "step": "cache_append(chunk) + chunk_attention(window)",
-        "l2": "flushed before every timed step (256 MiB write)",
+        "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
         "flops_convention": "absorbed MLA: 2*B*Nq*H*Nkv*(d_c+d_r+d_c) + append 2*B*Nq*224*1536",
     }
 
@@ -285,8 +287,15 @@ def run_ours(args, w, rank, world, local_rank):
                              w.grid_h, w.grid_w)
     x_chunk = x_all[:, w.n_cached:].contiguous()
     del x_all
-    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
+
+    class _Flush:
+        def zero_(self):
+            flush_w.zero_()          # evict: every L2 line now holds this (dirty) buffer
+            flush_r.max()            # read another buffer: the dirty lines are written back now
+    flush_buf = _Flush()
 
     def step():
         vm.vmla_cache_append(x_chunk, wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w, stream)

@@ -15,7 +15,10 @@
 // Tiling: a CTA owns 32 tokens x all 224 outputs; each of its 4 warps owns 8
 // tokens, and lane l owns outputs l + 32 i (i = 0..6), so the rope dims (outputs
 // 192..223) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
-// Operands are staged per 64-wide k chunk in shared memory as fp32.
+// Operands are staged per 64-wide k chunk in shared memory as fp32, double
+// buffered: the global loads of chunk c+1 are issued into registers before the
+// FMAs of chunk c, and land in the other buffer after them, so their latency
+// hides behind the arithmetic.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -30,7 +33,10 @@ constexpr int kThreads = 128;    // 4 warps
 constexpr int kTokPerWarp = 8;
 constexpr int kOutPerLane = 7;   // 224 / 32
 constexpr int kStride = kKc + 4; // fp32 row stride in shared memory (conflict-free float4 reads)
-constexpr int kSmemBytes = (kDrow + kTok) * kStride * 4;
+constexpr int kBufFloats = (kDrow + kTok) * kStride;
+constexpr int kSmemBytes = 2 * kBufFloats * 4;
+constexpr int kWVec = kDrow * 8 / kThreads;  // 16-byte W vectors per thread per chunk (14)
+constexpr int kXVec = kTok * 8 / kThreads;   // 16-byte x vectors per thread per chunk (2)
 
 struct AppendParams {
   const uint16_t* x;
@@ -67,30 +73,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < kOutPerLane; ++i) acc[t][i] = 0.0f;
 
-  for (int k0 = 0; k0 < p.d_model; k0 += kKc) {
-    __syncthreads();
-    for (int v = threadIdx.x; v < kDrow * 8; v += kThreads) {
-      const int n = v >> 3, kk = (v & 7) * 8;
-      const uint16_t* src = n < kDc ? p.w_dkv + (int64_t)n * p.d_model
-                                    : p.w_kr + (int64_t)(n - kDc) * p.d_model;
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + k0 + kk));
-      float4 lo, hi;
-      bf16x8_to_f32(u, lo, hi);
-      *reinterpret_cast<float4*>(ws + n * kStride + kk) = lo;
-      *reinterpret_cast<float4*>(ws + n * kStride + kk + 4) = hi;
+  // Register staging of one k chunk: vector v = threadIdx.x + kThreads * n.
+  uint4 wreg[kWVec], xreg[kXVec];
+  auto load_chunk = [&](int k0) {
+#pragma unroll
+    for (int n = 0; n < kWVec; ++n) {
+      const int v = threadIdx.x + kThreads * n;
+      const int row = v >> 3, kk = (v & 7) * 8;
+      const uint16_t* src = row < kDc ? p.w_dkv + (int64_t)row * p.d_model
+                                      : p.w_kr + (int64_t)(row - kDc) * p.d_model;
+      wreg[n] = __ldg(reinterpret_cast<const uint4*>(src + k0 + kk));
     }
-    for (int v = threadIdx.x; v < kTok * 8; v += kThreads) {
+#pragma unroll
+    for (int n = 0; n < kXVec; ++n) {
+      const int v = threadIdx.x + kThreads * n;
       const int t = v >> 3, kk = (v & 7) * 8;
-      float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
-      if (tok0 + t < p.n_tok) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)(tok0 + t) * p.d_model + k0 + kk));
-        bf16x8_to_f32(u, lo, hi);
-      }
+      xreg[n] = tok0 + t < p.n_tok
+                    ? __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)(tok0 + t) * p.d_model + k0 + kk))
+                    : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto store_chunk = [&](float* buf) {
+    float* ws = buf;
+    float* xs = buf + kDrow * kStride;
+#pragma unroll
+    for (int n = 0; n < kWVec; ++n) {
+      const int v = threadIdx.x + kThreads * n;
+      const int row = v >> 3, kk = (v & 7) * 8;
+      float4 lo, hi;
+      bf16x8_to_f32(wreg[n], lo, hi);
+      *reinterpret_cast<float4*>(ws + row * kStride + kk) = lo;
+      *reinterpret_cast<float4*>(ws + row * kStride + kk + 4) = hi;
+    }
+#pragma unroll
+    for (int n = 0; n < kXVec; ++n) {
+      const int v = threadIdx.x + kThreads * n;
+      const int t = v >> 3, kk = (v & 7) * 8;
+      float4 lo, hi;
+      bf16x8_to_f32(xreg[n], lo, hi);
       *reinterpret_cast<float4*>(xs + t * kStride + kk) = lo;
       *reinterpret_cast<float4*>(xs + t * kStride + kk + 4) = hi;
     }
-    __syncthreads();
-#pragma unroll 2
+  };
+
+  const int n_chunks = p.d_model / kKc;
+  load_chunk(0);
+  store_chunk(smem_f);
+  __syncthreads();
+  for (int c = 0; c < n_chunks; ++c) {
+    const float* ws = smem_f + (c & 1) * kBufFloats;
+    const float* xs = ws + kDrow * kStride;
+    if (c + 1 < n_chunks) load_chunk((c + 1) * kKc);
+#pragma unroll 1
     for (int kk = 0; kk < kKc; kk += 4) {
       float4 wv[kOutPerLane];
 #pragma unroll
@@ -110,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (c + 1 < n_chunks) store_chunk(smem_f + ((c + 1) & 1) * kBufFloats);
+    __syncthreads();
   }
 
   // 3D rotary embedding of the rope dims (output 192 + lane).
