@@ -122,6 +122,46 @@ vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uin
                                  int32_t d_head, float scale, uint16_t* out, void* stream);
 
 /*
+ * Non-absorbed form of the same attention (the latent cache stays the only cache).
+ * (abstract: per-head keys and values are generated from the head-shared content
+ * latent; summary "Approach".)  Per-head keys K_h = c . W_UK_h^T and values
+ * V_h = c . W_UV_h^T are materialised from the cache, then each query attends with
+ * the 160-dim key [K_h ; k_r] (k_r read from the cache) and the 128-dim value V_h.
+ * The result equals vmla_chunk_attention's up to rounding; the work per query, head
+ * and key is 2 x (160 + 128) FLOPs instead of 2 x (224 + 192), and the
+ * materialisation can be shared by every denoising step of a chunk.
+ *
+ * vmla_materialized_kv_bytes -- bytes of the materialised buffer kv[batch, n_kv, 2*heads, 128]
+ *   (bf16; heads [0, heads) hold K_h, heads [heads, 2*heads) hold V_h); 0 on bad sizes.
+ *
+ * vmla_materialize_kv -- writes kv (caller-owned, vmla_materialized_kv_bytes bytes) from
+ *   cache rows [0, n_kv) of cache[batch, cap, 224] and w_uk, w_uv [heads*128, 192].
+ *   bf16 tensor-core products, fp32 accumulation, bf16 rounding.  Limits: 1 <= n_kv <= cap < 2^31.
+ *
+ * vmla_chunk_attention_materialized -- out[batch, n_q, heads, 128] from q, q_rope (as for
+ *   vmla_chunk_attention), the materialised kv and the rope keys of cache rows [0, n_kv).
+ *
+ * vmla_chunk_attention_nonabsorbed -- both steps in one call; `workspace` (device,
+ *   16-byte aligned, >= vmla_materialized_kv_bytes(batch, heads, n_kv) bytes) receives kv.
+ */
+int64_t vmla_materialized_kv_bytes(int32_t batch, int32_t heads, int64_t n_kv);
+
+vmla_status vmla_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, const uint16_t* cache,
+                                int32_t batch, int32_t heads, int64_t cap, int64_t n_kv, uint16_t* kv,
+                                void* stream);
+
+vmla_status vmla_chunk_attention_materialized(const uint16_t* q, const uint16_t* q_rope, const uint16_t* kv,
+                                              const uint16_t* cache, int32_t batch, int32_t n_q, int32_t heads,
+                                              int64_t cap, int64_t n_kv, int64_t t0, int32_t grid_h,
+                                              int32_t grid_w, float scale, uint16_t* out, void* stream);
+
+vmla_status vmla_chunk_attention_nonabsorbed(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                             const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                             int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv, int64_t t0,
+                                             int32_t grid_h, int32_t grid_w, float scale, void* workspace,
+                                             int64_t workspace_bytes, uint16_t* out, void* stream);
+
+/*
  * vmla_get_device_status -- synchronises `stream`, then reports (and clears) any
  * wait timeout recorded by this library's kernels on the current device since the
  * last call: VMLA_ERR_TIMEOUT, VMLA_ERR_CUDA on a CUDA error, else VMLA_OK.

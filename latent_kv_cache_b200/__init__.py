@@ -52,6 +52,15 @@ def _load():
     lib.vmla_get_device_status.restype = ctypes.c_int
     lib.vmla_selftest_wait_timeout.argtypes = [i64, P]
     lib.vmla_selftest_wait_timeout.restype = ctypes.c_int
+    lib.vmla_materialized_kv_bytes.argtypes = [i32, i32, i64]
+    lib.vmla_materialized_kv_bytes.restype = i64
+    lib.vmla_materialize_kv.argtypes = [P, P, P, i32, i32, i64, i64, P, P]
+    lib.vmla_materialize_kv.restype = ctypes.c_int
+    lib.vmla_chunk_attention_materialized.argtypes = [P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32, P, P]
+    lib.vmla_chunk_attention_materialized.restype = ctypes.c_int
+    lib.vmla_chunk_attention_nonabsorbed.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32,
+                                                     P, i64, P, P]
+    lib.vmla_chunk_attention_nonabsorbed.restype = ctypes.c_int
     return lib
 
 
@@ -127,6 +136,53 @@ def vmla_dense_attention(q, k, v, scale: float, out, stream=None) -> None:
         raise ValueError("q/k/v/out shapes do not match")
     _check(lib.vmla_dense_attention(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), B, Nq, Nk, H, d,
                                     float(scale), _ptr(out, "out"), _stream(stream)))
+
+
+def _check_latent_shapes(q, q_rope, cache, out):
+    B, Nq, H, dh = q.shape
+    if dh != D_HEAD or tuple(q_rope.shape) != (B, Nq, H, D_R) or tuple(out.shape) != (B, Nq, H, D_HEAD):
+        raise ValueError("q/q_rope/out shapes do not match [B, Nq, H, 128|32]")
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D_C + D_R:
+        raise ValueError("cache must be [B, cap, 224]")
+    return B, Nq, H
+
+
+def vmla_materialized_kv_bytes(batch: int, heads: int, n_kv: int) -> int:
+    return int(lib.vmla_materialized_kv_bytes(int(batch), int(heads), int(n_kv)))
+
+
+def vmla_materialize_kv(w_uk, w_uv, cache, n_kv: int, kv, stream=None) -> None:
+    """kv [B, n_kv, 2H, 128]: K_h = c . W_UK_h^T in heads [0, H), V_h = c . W_UV_h^T in [H, 2H)."""
+    B, cap = cache.shape[0], cache.shape[1]
+    H = w_uk.shape[0] // D_HEAD
+    if tuple(kv.shape) != (B, n_kv, 2 * H, D_HEAD):
+        raise ValueError("kv must be [B, n_kv, 2H, 128]")
+    _check(lib.vmla_materialize_kv(_ptr(w_uk, "w_uk"), _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, H, cap,
+                                   int(n_kv), _ptr(kv, "kv"), _stream(stream)))
+
+
+def vmla_chunk_attention_materialized(q, q_rope, kv, cache, n_kv: int, t0: int, grid_h: int, grid_w: int,
+                                      scale: float, out, stream=None) -> None:
+    B, Nq, H = _check_latent_shapes(q, q_rope, cache, out)
+    if kv.dim() != 4 or kv.shape[0] != B or kv.shape[1] < n_kv or kv.shape[2] != 2 * H:
+        raise ValueError("kv must be [B, n_kv, 2H, 128]")
+    _check(lib.vmla_chunk_attention_materialized(_ptr(q, "q"), _ptr(q_rope, "q_rope"), _ptr(kv, "kv"),
+                                                 _ptr(cache, "cache"), B, Nq, H, cache.shape[1], int(n_kv), int(t0),
+                                                 int(grid_h), int(grid_w), float(scale), _ptr(out, "out"),
+                                                 _stream(stream)))
+
+
+def vmla_chunk_attention_nonabsorbed(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0: int, grid_h: int, grid_w: int,
+                                     scale: float, workspace, out, stream=None) -> None:
+    """workspace: a CUDA tensor of at least vmla_materialized_kv_bytes(B, H, n_kv) bytes."""
+    B, Nq, H = _check_latent_shapes(q, q_rope, cache, out)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check(lib.vmla_chunk_attention_nonabsorbed(_ptr(q, "q"), _ptr(q_rope, "q_rope"), _ptr(w_uk, "w_uk"),
+                                                _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, Nq, H, cache.shape[1],
+                                                int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
+                                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                                _ptr(out, "out"), _stream(stream)))
 
 
 def vmla_get_device_status(stream=None) -> None:

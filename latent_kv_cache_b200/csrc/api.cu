@@ -21,6 +21,13 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
                                    int n_q, int64_t n_kv, int heads, float scale, uint16_t* out,
                                    int* status, cudaStream_t stream, bool* encode_failed);
 cudaError_t launch_selftest_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t s);
+cudaError_t launch_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, const uint16_t* cache, int batch,
+                                  int heads, int64_t cap, int64_t n_kv, uint16_t* kv, int* status,
+                                  cudaStream_t stream, bool* encode_failed);
+cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* kv,
+                                 const uint16_t* cache, int batch, int n_q, int heads, int64_t cap,
+                                 int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale, uint16_t* out,
+                                 int* status, cudaStream_t stream, bool* encode_failed);
 }  // namespace vmla
 
 namespace {
@@ -141,6 +148,87 @@ vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uin
   if (enc_fail) return fail(VMLA_ERR_CUDA, "dense_attention: tensor-map encoding failed");
   if (e != cudaSuccess) return cuda_fail(e, "dense_attention launch");
   return VMLA_OK;
+}
+
+// Shared checks of the latent-attention arguments (chunk attention, both forms).
+static vmla_status check_latent_attention(const char* who, int32_t batch, int32_t n_q, int32_t heads, int64_t cap,
+                                          int64_t n_kv, int64_t t0, int32_t grid_h, int32_t grid_w, float scale) {
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "%s: batch must be in [1, 65535]", who);
+  if (n_q < 1) return fail(VMLA_ERR_INVALID_ARG, "%s: n_q must be >= 1", who);
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "%s: heads must be in [1, 512]", who);
+  if (n_kv < 1 || n_kv > cap) return fail(VMLA_ERR_INVALID_ARG, "%s: need 1 <= n_kv <= cap", who);
+  if (cap >= (int64_t(1) << 31)) return fail(VMLA_ERR_UNSUPPORTED, "%s: cap must be < 2^31", who);
+  if ((int64_t)((n_q + 127) / 128) * heads > 0x7FFFFFFF)
+    return fail(VMLA_ERR_UNSUPPORTED, "%s: too many query tiles", who);
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VMLA_ERR_INVALID_ARG, "%s: scale must be positive and finite", who);
+  return check_positions(n_q, t0, grid_h, grid_w);
+}
+
+int64_t vmla_materialized_kv_bytes(int32_t batch, int32_t heads, int64_t n_kv) {
+  if (batch < 1 || heads < 1 || n_kv < 1) return 0;
+  return (int64_t)batch * n_kv * 2 * heads * vmla::kDh * 2;
+}
+
+vmla_status vmla_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, const uint16_t* cache,
+                                int32_t batch, int32_t heads, int64_t cap, int64_t n_kv, uint16_t* kv,
+                                void* stream) {
+  if (!aligned16(w_uk) || !aligned16(w_uv) || !aligned16(cache) || !aligned16(kv))
+    return fail(VMLA_ERR_INVALID_ARG, "materialize_kv: pointers must be non-null and 16-byte aligned");
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "materialize_kv: batch must be in [1, 65535]");
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "materialize_kv: heads must be in [1, 512]");
+  if (n_kv < 1 || n_kv > cap) return fail(VMLA_ERR_INVALID_ARG, "materialize_kv: need 1 <= n_kv <= cap");
+  if (cap >= (int64_t(1) << 31)) return fail(VMLA_ERR_UNSUPPORTED, "materialize_kv: cap must be < 2^31");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "materialize_kv: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_materialize_kv(w_uk, w_uv, cache, batch, heads, cap, n_kv, kv, status,
+                                              static_cast<cudaStream_t>(stream), &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "materialize_kv: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "materialize_kv launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_chunk_attention_materialized(const uint16_t* q, const uint16_t* q_rope, const uint16_t* kv,
+                                              const uint16_t* cache, int32_t batch, int32_t n_q, int32_t heads,
+                                              int64_t cap, int64_t n_kv, int64_t t0, int32_t grid_h,
+                                              int32_t grid_w, float scale, uint16_t* out, void* stream) {
+  if (!aligned16(q) || !aligned16(q_rope) || !aligned16(kv) || !aligned16(cache) || !aligned16(out))
+    return fail(VMLA_ERR_INVALID_ARG,
+                "chunk_attention_materialized: pointers must be non-null and 16-byte aligned");
+  vmla_status st = check_latent_attention("chunk_attention_materialized", batch, n_q, heads, cap, n_kv, t0,
+                                          grid_h, grid_w, scale);
+  if (st != VMLA_OK) return st;
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "chunk_attention_materialized: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_mat_attention(q, q_rope, kv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
+                                             grid_w, scale, out, status, static_cast<cudaStream_t>(stream),
+                                             &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "chunk_attention_materialized: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention_materialized launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_chunk_attention_nonabsorbed(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                             const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                             int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv, int64_t t0,
+                                             int32_t grid_h, int32_t grid_w, float scale, void* workspace,
+                                             int64_t workspace_bytes, uint16_t* out, void* stream) {
+  if (!aligned16(workspace))
+    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention_nonabsorbed: workspace must be non-null and 16-byte aligned");
+  vmla_status st = check_latent_attention("chunk_attention_nonabsorbed", batch, n_q, heads, cap, n_kv, t0,
+                                          grid_h, grid_w, scale);
+  if (st != VMLA_OK) return st;
+  const int64_t need = vmla_materialized_kv_bytes(batch, heads, n_kv);
+  if (workspace_bytes < need)
+    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention_nonabsorbed: workspace of %lld bytes, need %lld",
+                (long long)workspace_bytes, (long long)need);
+  uint16_t* kv = static_cast<uint16_t*>(workspace);
+  st = vmla_materialize_kv(w_uk, w_uv, cache, batch, heads, cap, n_kv, kv, stream);
+  if (st != VMLA_OK) return st;
+  return vmla_chunk_attention_materialized(q, q_rope, kv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h, grid_w,
+                                           scale, out, stream);
 }
 
 vmla_status vmla_get_device_status(void* stream) {

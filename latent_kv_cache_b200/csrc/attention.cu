@@ -51,8 +51,14 @@ constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kBM = 128;                          // queries per tile
 constexpr uint32_t kTmemCols = 512;
 
+// Kernel variants: latent chunk attention with W_UK absorbed (kKindMla), the dense
+// per-head baseline (kKindDense), and attention over per-head keys/values
+// materialised from the latent cache (kKindMat: content keys and values from a
+// [B, n_kv, 2H, 128] buffer, the rope key straight from the latent cache).
+enum Kind : int { kKindMla = 0, kKindDense = 1, kKindMat = 2 };
+
 // Per-variant configuration.
-template <bool kMla>
+template <int kKind>
 struct Cfg;
 
 // MLA: the Qa operand (128 x 224 bf16) sits in shared memory (SS MMAs for the
@@ -60,7 +66,7 @@ struct Cfg;
 // 512 TMEM columns, and 128-key score tiles matter more than the A source
 // (a K = 16 tcgen05.mma takes at least ~93 cycles, so narrower N loses).
 template <>
-struct Cfg<true> {
+struct Cfg<kKindMla> {
   static constexpr int kBN = 128;                              // keys per tile
   static constexpr int kStages = 3;
   static constexpr uint32_t kBlkRows = 128 * 128;              // one 128B-swizzled block of a key tile
@@ -72,7 +78,7 @@ struct Cfg<true> {
 
 // Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
 template <>
-struct Cfg<false> {
+struct Cfg<kKindDense> {
   static constexpr int kBN = 128;
   static constexpr int kStages = 3;
   static constexpr uint32_t kBlkRows = 128 * 128;
@@ -82,24 +88,38 @@ struct Cfg<false> {
   static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
 };
 
+// Materialised keys/values: Q = [q_h ; RoPE(q_r)] (80 cells) in TMEM; key tile =
+// [content 128 ; rope 32], value tile 128.
+template <>
+struct Cfg<kKindMat> {
+  static constexpr int kBN = 128;
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kBlkRows = 128 * 128;
+  static constexpr uint32_t kStage = 4 * kBlkRows + 128 * 64;  // [K: 2 | V: 2 blocks | k_r] = 73728
+  static constexpr uint32_t kQaBytes = 0;
+  static constexpr int kOCols = kDh;
+  static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
+};
+
 constexpr uint32_t kBlk128 = 128 * 128;  // 128 rows x 128 B: prologue / epilogue operand blocks
 constexpr uint32_t kTmemO = 0;
 
-template <bool kMla>
+template <int kKind>
 struct Layout {
-  static constexpr uint32_t kRingOff = Cfg<kMla>::kQaBytes;
-  static constexpr uint32_t kBarOff = kRingOff + Cfg<kMla>::kStages * Cfg<kMla>::kStage;
+  static constexpr uint32_t kRingOff = Cfg<kKind>::kQaBytes;
+  static constexpr uint32_t kBarOff = kRingOff + Cfg<kKind>::kStages * Cfg<kKind>::kStage;
   static constexpr uint32_t kRedOff = kBarOff + 512;
   static constexpr uint32_t kUsed = kRedOff + 2 * 2 * 128 * 4;
   static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
   static constexpr uint32_t kMaxPad = kBytes - kUsed;  // alignment slack the kernel checks for
 };
-static_assert(Layout<true>::kBytes <= 232448, "MLA shared memory");
-static_assert(Layout<false>::kBytes <= 232448, "dense shared memory");
-static_assert(Layout<true>::kMaxPad >= 512 && Layout<false>::kMaxPad >= 512, "alignment slack");
+static_assert(Layout<kKindMla>::kBytes <= 232448 && Layout<kKindDense>::kBytes <= 232448 &&
+              Layout<kKindMat>::kBytes <= 232448, "shared memory");
+static_assert(Layout<kKindMla>::kMaxPad >= 512 && Layout<kKindDense>::kMaxPad >= 512 &&
+              Layout<kKindMat>::kMaxPad >= 512, "alignment slack");
 // The MLA prologue parks q (2 blocks) and W_UK (3 blocks) in the first ring stages.
-static_assert(5 * kBlk128 <= 2 * Cfg<true>::kStage, "prologue operands fit in stages 0-1");
-static_assert(2 * kBlk128 <= Cfg<true>::kStage && kBlk128 <= Cfg<true>::kStage, "W_UV blocks fit");
+static_assert(5 * kBlk128 <= 2 * Cfg<kKindMla>::kStage, "prologue operands fit in stages 0-1");
+static_assert(2 * kBlk128 <= Cfg<kKindMla>::kStage && kBlk128 <= Cfg<kKindMla>::kStage, "W_UV blocks fit");
 
 enum Bar {
   B_PRO = 0, B_QABS, B_QA,
@@ -124,6 +144,12 @@ struct ChunkMaps {
 struct DenseMaps {
   CUtensorMap k;  // [B, Nk, H, 128] box (64, 1, 128, 1)
   CUtensorMap v;  // [B, Nk, H, 128]
+};
+
+struct MatMaps {
+  CUtensorMap k;   // [B, n_kv, 2H, 128] box (64, 1, 128, 1): heads [0, H) keys, [H, 2H) values
+  CUtensorMap v;   // same tensor (values addressed at head H + h)
+  CUtensorMap kr;  // latent cache [B, n_kv, 224] box (32, 128, 1), 64B swizzle (rope key, x = 192)
 };
 
 struct AttnParams {
@@ -204,11 +230,11 @@ __device__ __forceinline__ bool exchange(const SoftmaxThread& t, uint32_t bars, 
 }
 
 // Softmax step for key tile j.  Returns false on abort.
-template <bool kMla>
+template <int kKind>
 __device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const SoftmaxThread& t,
                                              const AttnParams& p, const WaitCtl& ctl,
                                              float& m_run, float& l_part) {
-  using C = Cfg<kMla>;
+  using C = Cfg<kKind>;
   constexpr int kW = C::kBN / 2;  // score columns per thread (48 or 64)
   const int sb = j & 1;
   if (!warp_wait(bar_addr(bars, B_SF0 + sb), (j >> 1) & 1, ctl)) return false;
@@ -296,14 +322,49 @@ __device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const Softmax
   return true;
 }
 
+// Rope part of query qi of head h, rotated with the query's own (t, row, col);
+// zeros for padding rows (qi >= n_q).
+__device__ __forceinline__ void rope_query(const AttnParams& p, const RopeTable* tab, int b, int qi, int h,
+                                           float (&qr)[kDr]) {
+#pragma unroll
+  for (int e = 0; e < kDr; ++e) qr[e] = 0.0f;
+  if (qi >= p.n_q) return;
+  const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDr);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 u = __ldg(src + c);
+    qr[8 * c + 0] = bf16lo_to_f32(u.x); qr[8 * c + 1] = bf16hi_to_f32(u.x);
+    qr[8 * c + 2] = bf16lo_to_f32(u.y); qr[8 * c + 3] = bf16hi_to_f32(u.y);
+    qr[8 * c + 4] = bf16lo_to_f32(u.z); qr[8 * c + 5] = bf16hi_to_f32(u.z);
+    qr[8 * c + 6] = bf16lo_to_f32(u.w); qr[8 * c + 7] = bf16hi_to_f32(u.w);
+  }
+  const int per_frame = p.grid_h * p.grid_w;
+  const int f = qi / per_frame;
+  const int rem = qi - f * per_frame;
+  const int row = rem / p.grid_w;
+  const int col = rem - row * p.grid_w;
+#pragma unroll
+  for (int pr = 0; pr < kDr / 2; ++pr) {
+    float2 cs;
+    if (pr < kPairsT) cs = tab->t[f][pr];
+    else if (pr < kPairsT + kPairsH) cs = tab->h[row][pr - kPairsT];
+    else cs = tab->w[col][pr - kPairsT - kPairsH];
+    const float a = qr[2 * pr], bb = qr[2 * pr + 1];
+    qr[2 * pr] = a * cs.x - bb * cs.y;
+    qr[2 * pr + 1] = a * cs.y + bb * cs.x;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // The attention kernel.  kMla: latent chunk attention (absorbed W_UK, [c ; k_r]
 // tiles, W_UV epilogue); otherwise the dense per-head baseline (d = 128).
 // ---------------------------------------------------------------------------
-template <bool kMla, class Maps>
+template <int kKind, class Maps>
 __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p, const RopeTable* tab) {
-  using C = Cfg<kMla>;
-  using L = Layout<kMla>;
+  constexpr bool kMla = kKind == kKindMla;
+  constexpr bool kMat = kKind == kKindMat;
+  using C = Cfg<kKind>;
+  using L = Layout<kKind>;
   constexpr int kBN = C::kBN;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kStage = C::kStage;
@@ -382,6 +443,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       } else {
         tma_prefetch_desc(&maps.k);
         tma_prefetch_desc(&maps.v);
+        if constexpr (kMat) tma_prefetch_desc(&maps.kr);
       }
       // MLA: n_tiles key tiles, then W_UV_h blocks {0,1} and {2} as two more ring items.
       const int n_items = kMla ? n_tiles + 2 : n_tiles;
@@ -412,11 +474,13 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             tma_load_2d(sa, &maps.wuv, fb, 128, h * kDh);
           }
         } else {
+          const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
           mbar_arrive_expect_tx(fb, kStage);
           tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
           tma_load_4d(sa + C::kBlkRows, &maps.k, fb, 64, h, kv0, b);
-          tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, h, kv0, b);
-          tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, h, kv0, b);
+          tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, hv, kv0, b);
+          tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, hv, kv0, b);
+          if constexpr (kMat) tma_load_3d(sa + 4 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
         }
         last_use[st] = use;
       }
@@ -484,9 +548,13 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
           }
         } else {
+          // S = Q . K^T with Q from TMEM: 8 steps over the 128B-swizzled content key
+          // blocks (+2 over the 64B-swizzled rope block for the materialised variant).
+          constexpr int kSteps = kMat ? 10 : 8;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t bd = smem_desc(sa + (k >> 2) * C::kBlkRows + (k & 3) * 32, 16, 1024, kSw128);
+          for (int k = 0; k < kSteps; ++k) {
+            const uint64_t bd = k < 8 ? smem_desc(sa + (k >> 2) * C::kBlkRows + (k & 3) * 32, 16, 1024, kSw128)
+                                      : smem_desc(sa + 4 * C::kBlkRows + (k - 8) * 32, 16, 512, kSw64);
             umma_ts(d, tmem + C::kTmemQ + k * 8, bd, kIdS, k > 0);
           }
         }
@@ -545,37 +613,8 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             st_sw128_chunk(smem + (col >> 6) * C::kBlkRows, t.r, ((col & 63) >> 3) + q4, pack8(v + 8 * q4, 1.0f));
         }
         if (t.half == 0) {
-          // Rope part of the query, rotated with the query's own (t, row, col).
           float qr[kDr];
-#pragma unroll
-          for (int e = 0; e < kDr; ++e) qr[e] = 0.0f;
-          if (qi < p.n_q) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                p.q_rope + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDr);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 u = __ldg(src + c);
-              qr[8 * c + 0] = bf16lo_to_f32(u.x); qr[8 * c + 1] = bf16hi_to_f32(u.x);
-              qr[8 * c + 2] = bf16lo_to_f32(u.y); qr[8 * c + 3] = bf16hi_to_f32(u.y);
-              qr[8 * c + 4] = bf16lo_to_f32(u.z); qr[8 * c + 5] = bf16hi_to_f32(u.z);
-              qr[8 * c + 6] = bf16lo_to_f32(u.w); qr[8 * c + 7] = bf16hi_to_f32(u.w);
-            }
-            const int per_frame = p.grid_h * p.grid_w;
-            const int f = qi / per_frame;
-            const int rem = qi - f * per_frame;
-            const int row = rem / p.grid_w;
-            const int col = rem - row * p.grid_w;
-#pragma unroll
-            for (int pr = 0; pr < kDr / 2; ++pr) {
-              float2 cs;
-              if (pr < kPairsT) cs = tab->t[f][pr];
-              else if (pr < kPairsT + kPairsH) cs = tab->h[row][pr - kPairsT];
-              else cs = tab->w[col][pr - kPairsT - kPairsH];
-              const float a = qr[2 * pr], bb = qr[2 * pr + 1];
-              qr[2 * pr] = a * cs.x - bb * cs.y;
-              qr[2 * pr + 1] = a * cs.y + bb * cs.x;
-            }
-          }
+          rope_query(p, tab, b, qi, h, qr);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint4 w;
@@ -603,6 +642,16 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         }
       }
       tmem_st32(t.t_row + C::kTmemQ + 32 * t.half, v);
+      if constexpr (kMat) {
+        if (t.half == 0) {
+          float qr[kDr];
+          rope_query(p, tab, b, qi, h, qr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(qr[2 * e], qr[2 * e + 1]);
+          tmem_st16(t.t_row + C::kTmemQ + 64, pk);
+        }
+      }
     }
     if (ok) {
       tmem_st_wait();
@@ -610,7 +659,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       mbar_arrive(bar_addr(bars, B_QA));
     }
     float m_run = -INFINITY, l_part = 0.0f;
-    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kMla>(j, bars, t, p, ctl, m_run, l_part);
+    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kKind>(j, bars, t, p, ctl, m_run, l_part);
     float l_other = 0.0f;
     if (ok) ok = exchange(t, bars, n_tiles, l_part, l_other, ctl);
     if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
@@ -674,12 +723,18 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
 __global__ void __launch_bounds__(kThreads, 1)
     k_chunk_attn(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
                  const __grid_constant__ RopeTable tab) {
-  attn_body<true>(maps, p, &tab);
+  attn_body<kKindMla>(maps, p, &tab);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_dense_attn(const __grid_constant__ DenseMaps maps, const __grid_constant__ AttnParams p) {
-  attn_body<false>(maps, p, nullptr);
+  attn_body<kKindDense>(maps, p, nullptr);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_mat_attn(const __grid_constant__ MatMaps maps, const __grid_constant__ AttnParams p,
+               const __grid_constant__ RopeTable tab) {
+  attn_body<kKindMat>(maps, p, &tab);
 }
 
 // ---------------------------------------------------------------------------
@@ -744,7 +799,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
                                    cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_chunk_attn, Layout<true>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  if (!set_smem_attr((const void*)k_chunk_attn, Layout<kKindMla>::kBytes, attr_done)) return cudaErrorInvalidValue;
   ChunkMaps maps;
   bool ok = make_head_map(&maps.q, q, batch, n_q, heads);
   {
@@ -757,8 +812,8 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   {
     const cuuint64_t dims[3] = {(cuuint64_t)kDrow, (cuuint64_t)n_kv, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)kDrow * 2, (cuuint64_t)cap * kDrow * 2};
-    const cuuint32_t box_c[3] = {64, (cuuint32_t)Cfg<true>::kBN, 1};
-    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<true>::kBN, 1};
+    const cuuint32_t box_c[3] = {64, (cuuint32_t)Cfg<kKindMla>::kBN, 1};
+    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<kKindMla>::kBN, 1};
     ok = ok && make_map(&maps.c, cache, 3, dims, strides, box_c, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&maps.kr, cache, 3, dims, strides, box_r, CU_TENSOR_MAP_SWIZZLE_64B);
   }
@@ -775,7 +830,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + Cfg<true>::kBN - 1) / Cfg<true>::kBN);
+  p.n_kv_tiles = (int)((n_kv + Cfg<kKindMla>::kBN - 1) / Cfg<kKindMla>::kBN);
   p.grid_h = grid_h;
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -783,7 +838,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_chunk_attn<<<grid, kThreads, Layout<true>::kBytes, stream>>>(maps, p, tab);
+  k_chunk_attn<<<grid, kThreads, Layout<kKindMla>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 
@@ -792,7 +847,7 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
                                    int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_dense_attn, Layout<false>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  if (!set_smem_attr((const void*)k_dense_attn, Layout<kKindDense>::kBytes, attr_done)) return cudaErrorInvalidValue;
   DenseMaps maps;
   bool ok = make_head_map(&maps.k, k, batch, n_kv, heads) && make_head_map(&maps.v, v, batch, n_kv, heads);
   if (!ok) {
@@ -807,10 +862,50 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + Cfg<false>::kBN - 1) / Cfg<false>::kBN);
+  p.n_kv_tiles = (int)((n_kv + Cfg<kKindDense>::kBN - 1) / Cfg<kKindDense>::kBN);
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_dense_attn<<<grid, kThreads, Layout<false>::kBytes, stream>>>(maps, p);
+  k_dense_attn<<<grid, kThreads, Layout<kKindDense>::kBytes, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* kv,
+                                 const uint16_t* cache, int batch, int n_q, int heads, int64_t cap,
+                                 int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale, uint16_t* out,
+                                 int* status, cudaStream_t stream, bool* encode_failed) {
+  static bool attr_done[64] = {false};
+  *encode_failed = false;
+  if (!set_smem_attr((const void*)k_mat_attn, Layout<kKindMat>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  MatMaps maps;
+  bool ok = make_head_map(&maps.k, kv, batch, n_kv, 2 * heads) && make_head_map(&maps.v, kv, batch, n_kv, 2 * heads);
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)kDrow, (cuuint64_t)n_kv, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDrow * 2, (cuuint64_t)cap * kDrow * 2};
+    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<kKindMat>::kBN, 1};
+    ok = ok && make_map(&maps.kr, cache, 3, dims, strides, box_r, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  if (!ok) {
+    *encode_failed = true;
+    return cudaErrorInvalidValue;
+  }
+  AttnParams p{};
+  p.q = q;
+  p.q_rope = q_rope;
+  p.out = out;
+  p.status = status;
+  p.wait_limit_ns = kWaitLimitNs;
+  p.n_kv = n_kv;
+  p.n_q = n_q;
+  p.heads = heads;
+  p.n_kv_tiles = (int)((n_kv + Cfg<kKindMat>::kBN - 1) / Cfg<kKindMat>::kBN);
+  p.grid_h = grid_h;
+  p.grid_w = grid_w;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  static thread_local RopeTable tab;
+  const int per_frame = grid_h * grid_w;
+  build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
+  dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
+  k_mat_attn<<<grid, kThreads, Layout<kKindMat>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 

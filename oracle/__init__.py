@@ -241,6 +241,26 @@ def chunk_attention(q_bits, q_rope_bits, w_uk_bits, w_uv_bits, cache_bits, n_kv:
     return out
 
 
+def materialized_kv(w_uk_bits, w_uv_bits, cache_bits, n_kv: int) -> np.ndarray:
+    """Per-head content keys and values of cache rows [0, n_kv), float64
+    [B, n_kv, 2H, d_h]: heads [0, H) hold K_h = C . W_UK_h^T, heads [H, 2H) hold
+    V_h = C . W_UV_h^T (the non-absorbed keys/values of the abstract's shared latent)."""
+    wuk = decode_bf16(w_uk_bits)
+    wuv = decode_bf16(w_uv_bits)
+    cache = decode_bf16(cache_bits)
+    if cache.ndim == 2:
+        cache = cache[None]
+    d_c = wuk.shape[1]
+    dh = 128
+    H = wuk.shape[0] // dh
+    C = cache[:, :n_kv, :d_c]
+    out = np.empty((cache.shape[0], n_kv, 2 * H, dh), dtype=np.float64)
+    for h in range(H):
+        out[:, :, h] = C @ wuk[h * dh:(h + 1) * dh].T
+        out[:, :, H + h] = C @ wuv[h * dh:(h + 1) * dh].T
+    return out
+
+
 def chunk_attention_absorbed(q_bits, q_rope_bits, w_uk_bits, w_uv_bits, cache_bits, n_kv: int,
                              t0: int, grid_h: int, grid_w: int, scale: float, rows=None,
                              split=ROPE_SPLIT, theta=ROPE_THETA) -> np.ndarray:

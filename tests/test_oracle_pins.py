@@ -287,6 +287,26 @@ def test_absorbed_equals_nonabsorbed():
     assert np.linalg.norm(a - b) <= 1e-12 * np.linalg.norm(a)
 
 
+def test_materialized_kv_reproduces_attention():
+    # softmax over [K_h ; k_r] with the materialised K_h, V_h (torch SDPA, fp64) equals
+    # the absorbed formulation -- pins materialized_kv's head layout and transposes.
+    rng = np.random.default_rng(19)
+    B, Nq, n_kv, H, d_c, gh, gw, t0 = 2, 12, 30, 3, 20, 2, 3, 5
+    q, qr, wuk, wuv, cache = _tiny_case(rng, B, Nq, n_kv, H, 128, d_c, cap=33, gh=gh, gw=gw)
+    kv = oracle.materialized_kv(wuk, wuv, cache, n_kv)
+    assert kv.shape == (B, n_kv, 2 * H, 128)
+    ref = oracle.chunk_attention_absorbed(q, qr, wuk, wuv, cache, n_kv, t0, gh, gw, 0.3)
+    Q, QR, C = (torch.from_numpy(oracle.decode_bf16(a)) for a in (q, qr, cache))
+    t, r, c = oracle.token_positions(Nq, t0, gh, gw)
+    for h in range(H):
+        qrot = torch.from_numpy(oracle.rope3d(QR[:, :, h].numpy(), t, r, c))
+        Qh = torch.cat([Q[:, :, h], qrot], dim=-1)
+        Kh = torch.cat([torch.from_numpy(kv[:, :, h]), C[:, :n_kv, d_c:]], dim=-1)
+        Vh = torch.from_numpy(kv[:, :, H + h])
+        got = torch.nn.functional.scaled_dot_product_attention(Qh, Kh, Vh, scale=0.3)
+        np.testing.assert_allclose(got.numpy(), ref[:, :, h], rtol=1e-11, atol=1e-12)
+
+
 def test_attention_matches_torch_sdpa():
     rng = np.random.default_rng(11)
     B, Nq, n_kv, H, dh, d_c, gh, gw, t0 = 2, 24, 40, 3, 16, 24, 2, 4, 9

@@ -100,6 +100,10 @@ class Workload:
         """Query absorption (q_h . W_UK_h) and the W_UV epilogue of one call."""
         return 2.0 * 2.0 * self.batch * self.n_q * self.heads * self.d_head * self.d_c
 
+    def nonabsorbed_flops(self) -> float:
+        """Attention over materialised per-head keys [K_h ; k_r] (160) and values V_h (128)."""
+        return 2.0 * self.batch * self.n_q * self.heads * self.n_kv * (self.d_head + self.d_r + self.d_head)
+
     def dense_flops(self) -> float:
         """Dense per-head attention FLOPs (QK^T and PV, d = 128)."""
         return 2.0 * 2.0 * self.batch * self.n_q * self.heads * self.n_kv * self.d_head
