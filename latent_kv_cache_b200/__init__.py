@@ -34,7 +34,7 @@ class VmlaError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m latent_kv_cache_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python latent_kv_cache_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.c_void_p
     i32, i64, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_float

@@ -1,6 +1,8 @@
 """Build libvideomla.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m latent_kv_cache_b200.build [--force] [--verbose]
+    python latent_kv_cache_b200/build.py [--force] [--verbose]
+
+(Run it by path: importing the package first would load the shared library it builds.)
 
 Each .cu under csrc/ is compiled to an object in _build/ (in parallel), then
 linked into latent_kv_cache_b200/libvideomla.so with the static CUDA runtime.

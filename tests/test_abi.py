@@ -15,8 +15,8 @@ HEADER = os.path.join(ROOT, "include", "videomla.h")
 
 @pytest.fixture(scope="module")
 def vm():
-    from latent_kv_cache_b200 import build as b
-    b.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import latent_kv_cache_b200 as vm
     return vm
 
