@@ -162,6 +162,32 @@ vmla_status vmla_chunk_attention_nonabsorbed(const uint16_t* q, const uint16_t* 
                                              int64_t workspace_bytes, uint16_t* out, void* stream);
 
 /*
+ * vmla_chunk_attention_nonabsorbed_noalloc -- vmla_chunk_attention_nonabsorbed without
+ * a caller workspace: the library's own fixed scratch holds the materialised keys and
+ * values.  (No counterpart in the paper: this is an interface for callers that cannot
+ * allocate device memory -- for example a host program that only receives tensors from
+ * another runtime, a framework whose allocator already owns the device memory budget,
+ * or a loop that cannot take the device-wide synchronisation cudaMalloc/cudaFree imply.)
+ *
+ * Arguments and result are those of vmla_chunk_attention_nonabsorbed.  The scratch is a
+ * static device array of VMLA_NOALLOC_SCRATCH_BYTES that every GPU loading the library
+ * keeps until exit; sizes with vmla_materialized_kv_bytes(batch, heads, n_kv) above it
+ * return VMLA_ERR_UNSUPPORTED (use the workspace form).  The call allocates nothing.
+ * Its first call on a device looks up the scratch's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream
+ * capture.  All calls on a device share the one scratch and it keeps the last call's
+ * contents (nothing in it needs to start at zero), so calls that overlap on the GPU
+ * -- e.g. on two streams at once -- race with each other and must be serialised.
+ */
+#define VMLA_NOALLOC_SCRATCH_BYTES (8ll << 20)
+vmla_status vmla_chunk_attention_nonabsorbed_noalloc(const uint16_t* q, const uint16_t* q_rope,
+                                                     const uint16_t* w_uk, const uint16_t* w_uv,
+                                                     const uint16_t* cache, int32_t batch, int32_t n_q,
+                                                     int32_t heads, int64_t cap, int64_t n_kv, int64_t t0,
+                                                     int32_t grid_h, int32_t grid_w, float scale, uint16_t* out,
+                                                     void* stream);
+
+/*
  * vmla_get_device_status -- synchronises `stream`, then reports (and clears) any
  * wait timeout recorded by this library's kernels on the current device since the
  * last call: VMLA_ERR_TIMEOUT, VMLA_ERR_CUDA on a CUDA error, else VMLA_OK.

@@ -61,6 +61,9 @@ def _load():
     lib.vmla_chunk_attention_nonabsorbed.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32,
                                                      P, i64, P, P]
     lib.vmla_chunk_attention_nonabsorbed.restype = ctypes.c_int
+    lib.vmla_chunk_attention_nonabsorbed_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32,
+                                                             f32, P, P]
+    lib.vmla_chunk_attention_nonabsorbed_noalloc.restype = ctypes.c_int
     return lib
 
 
@@ -183,6 +186,21 @@ def vmla_chunk_attention_nonabsorbed(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0
                                                 int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
                                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                                 _ptr(out, "out"), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def vmla_chunk_attention_nonabsorbed_noalloc(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0: int, grid_h: int,
+                                             grid_w: int, scale: float, out, stream=None) -> None:
+    """Like vmla_chunk_attention_nonabsorbed, with the library's fixed scratch instead of a
+    workspace (for callers that cannot allocate device memory); calls must not overlap."""
+    B, Nq, H = _check_latent_shapes(q, q_rope, cache, out)
+    _check(lib.vmla_chunk_attention_nonabsorbed_noalloc(_ptr(q, "q"), _ptr(q_rope, "q_rope"), _ptr(w_uk, "w_uk"),
+                                                        _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, Nq, H,
+                                                        cache.shape[1], int(n_kv), int(t0), int(grid_h),
+                                                        int(grid_w), float(scale), _ptr(out, "out"),
+                                                        _stream(stream)))
 
 
 def vmla_get_device_status(stream=None) -> None:

@@ -62,6 +62,11 @@ vmla_status check_positions(int64_t n_tok, int64_t t0, int32_t grid_h, int32_t g
 
 }  // namespace
 
+namespace vmla {
+// Sets the calling thread's vmla_last_error() message (for entry points in other files).
+vmla_status record_error(vmla_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace vmla
+
 extern "C" {
 
 const char* vmla_status_string(int status) {
