@@ -122,6 +122,28 @@ vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uin
                                  int32_t d_head, float scale, uint16_t* out, void* stream);
 
 /*
+ * The projections either side of the attention (summary "Approach": the latent
+ * attention block of the Wan2.1 backbone; the pages give no formulas, these are the
+ * standard linear maps).  bf16 tensor-core GEMMs with fp32 accumulation, bf16 out.
+ *
+ * vmla_query_projection -- one pass over the hidden states x[batch, n_tok, d_model]:
+ *   q      [batch, n_tok, heads, 128] = x . W_Q^T,  w_q  [heads*128, d_model]
+ *   q_rope [batch, n_tok, heads, 32]  = x . W_QR^T, w_qr [heads*32, d_model]
+ *   (q_rope is left unrotated: vmla_chunk_attention rotates it with the token positions.)
+ *   Limits: d_model a multiple of 64; batch*n_tok < 2^31.
+ *
+ * vmla_output_projection -- y[batch, n_tok, d_model] = o . W_O^T with o the attention
+ *   output [batch, n_tok, heads, 128] and w_o [d_model, heads*128].
+ *   Limits: d_model a multiple of 128; batch*n_tok < 2^31.
+ */
+vmla_status vmla_query_projection(const uint16_t* x, const uint16_t* w_q, const uint16_t* w_qr, int32_t batch,
+                                  int32_t n_tok, int32_t d_model, int32_t heads, uint16_t* q, uint16_t* q_rope,
+                                  void* stream);
+
+vmla_status vmla_output_projection(const uint16_t* o, const uint16_t* w_o, int32_t batch, int32_t n_tok,
+                                   int32_t heads, int32_t d_model, uint16_t* y, void* stream);
+
+/*
  * Non-absorbed form of the same attention (the latent cache stays the only cache).
  * (abstract: per-head keys and values are generated from the head-shared content
  * latent; summary "Approach".)  Per-head keys K_h = c . W_UK_h^T and values

@@ -61,6 +61,10 @@ def _load():
     lib.vmla_chunk_attention_nonabsorbed.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32,
                                                      P, i64, P, P]
     lib.vmla_chunk_attention_nonabsorbed.restype = ctypes.c_int
+    lib.vmla_query_projection.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P]
+    lib.vmla_query_projection.restype = ctypes.c_int
+    lib.vmla_output_projection.argtypes = [P, P, i32, i32, i32, i32, P, P]
+    lib.vmla_output_projection.restype = ctypes.c_int
     lib.vmla_chunk_attention_nonabsorbed_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32,
                                                              f32, P, P]
     lib.vmla_chunk_attention_nonabsorbed_noalloc.restype = ctypes.c_int
@@ -139,6 +143,27 @@ def vmla_dense_attention(q, k, v, scale: float, out, stream=None) -> None:
         raise ValueError("q/k/v/out shapes do not match")
     _check(lib.vmla_dense_attention(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), B, Nq, Nk, H, d,
                                     float(scale), _ptr(out, "out"), _stream(stream)))
+
+
+def vmla_query_projection(x, w_q, w_qr, q, q_rope, stream=None) -> None:
+    """x [B, n, D] -> q [B, n, H, 128] = x W_Q^T and q_rope [B, n, H, 32] = x W_QR^T (unrotated)."""
+    B, n, D = x.shape
+    H = q.shape[2]
+    if tuple(q.shape) != (B, n, H, D_HEAD) or tuple(q_rope.shape) != (B, n, H, D_R):
+        raise ValueError("q must be [B, n, H, 128] and q_rope [B, n, H, 32]")
+    if tuple(w_q.shape) != (H * D_HEAD, D) or tuple(w_qr.shape) != (H * D_R, D):
+        raise ValueError("w_q must be [H*128, D] and w_qr [H*32, D]")
+    _check(lib.vmla_query_projection(_ptr(x, "x"), _ptr(w_q, "w_q"), _ptr(w_qr, "w_qr"), B, n, D, H,
+                                     _ptr(q, "q"), _ptr(q_rope, "q_rope"), _stream(stream)))
+
+
+def vmla_output_projection(o, w_o, y, stream=None) -> None:
+    """o [B, n, H, 128] -> y [B, n, D] = o W_O^T with w_o [D, H*128]."""
+    B, n, H, dh = o.shape
+    D = y.shape[2]
+    if dh != D_HEAD or tuple(y.shape) != (B, n, D) or tuple(w_o.shape) != (D, H * D_HEAD):
+        raise ValueError("o must be [B, n, H, 128], w_o [D, H*128], y [B, n, D]")
+    _check(lib.vmla_output_projection(_ptr(o, "o"), _ptr(w_o, "w_o"), B, n, H, D, _ptr(y, "y"), _stream(stream)))
 
 
 def _check_latent_shapes(q, q_rope, cache, out):

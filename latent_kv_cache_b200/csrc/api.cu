@@ -24,6 +24,9 @@ cudaError_t launch_selftest_wait_timeout(int* status, uint64_t limit_ns, cudaStr
 cudaError_t launch_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, const uint16_t* cache, int batch,
                                   int heads, int64_t cap, int64_t n_kv, uint16_t* kv, int* status,
                                   cudaStream_t stream, bool* encode_failed);
+cudaError_t launch_gemm_pair(const uint16_t* a, const uint16_t* b0, const uint16_t* b1, int m, int n0, int n1,
+                             int k, uint16_t* c0, int64_t ldc0, uint16_t* c1, int64_t ldc1, int* status,
+                             cudaStream_t stream, bool* encode_failed);
 cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* kv,
                                  const uint16_t* cache, int batch, int n_q, int heads, int64_t cap,
                                  int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale, uint16_t* out,
@@ -234,6 +237,47 @@ vmla_status vmla_chunk_attention_nonabsorbed(const uint16_t* q, const uint16_t* 
   if (st != VMLA_OK) return st;
   return vmla_chunk_attention_materialized(q, q_rope, kv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h, grid_w,
                                            scale, out, stream);
+}
+
+vmla_status vmla_query_projection(const uint16_t* x, const uint16_t* w_q, const uint16_t* w_qr, int32_t batch,
+                                  int32_t n_tok, int32_t d_model, int32_t heads, uint16_t* q, uint16_t* q_rope,
+                                  void* stream) {
+  if (!aligned16(x) || !aligned16(w_q) || !aligned16(w_qr) || !aligned16(q) || !aligned16(q_rope))
+    return fail(VMLA_ERR_INVALID_ARG, "query_projection: pointers must be non-null and 16-byte aligned");
+  if (batch < 1 || n_tok < 1 || (int64_t)batch * n_tok > 0x7FFFFFFF)
+    return fail(VMLA_ERR_INVALID_ARG, "query_projection: need batch, n_tok >= 1 and batch*n_tok < 2^31");
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "query_projection: heads must be in [1, 512]");
+  if (d_model < 64 || d_model > 65536 || d_model % 64 != 0)
+    return fail(VMLA_ERR_UNSUPPORTED, "query_projection: d_model must be a multiple of 64 in [64, 65536]");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "query_projection: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_gemm_pair(x, w_q, w_qr, batch * n_tok, heads * vmla::kDh, heads * vmla::kDr, d_model,
+                                         q, (int64_t)heads * vmla::kDh, q_rope, (int64_t)heads * vmla::kDr, status,
+                                         static_cast<cudaStream_t>(stream), &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "query_projection: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "query_projection launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_output_projection(const uint16_t* o, const uint16_t* w_o, int32_t batch, int32_t n_tok,
+                                   int32_t heads, int32_t d_model, uint16_t* y, void* stream) {
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(y))
+    return fail(VMLA_ERR_INVALID_ARG, "output_projection: pointers must be non-null and 16-byte aligned");
+  if (batch < 1 || n_tok < 1 || (int64_t)batch * n_tok > 0x7FFFFFFF)
+    return fail(VMLA_ERR_INVALID_ARG, "output_projection: need batch, n_tok >= 1 and batch*n_tok < 2^31");
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "output_projection: heads must be in [1, 512]");
+  if (d_model < 128 || d_model > 65536 || d_model % 128 != 0)
+    return fail(VMLA_ERR_UNSUPPORTED, "output_projection: d_model must be a multiple of 128 in [128, 65536]");
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "output_projection: no CUDA device");
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_gemm_pair(o, w_o, nullptr, batch * n_tok, d_model, 0, heads * vmla::kDh, y,
+                                         (int64_t)d_model, nullptr, 0, status, static_cast<cudaStream_t>(stream),
+                                         &enc_fail);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "output_projection: tensor-map encoding failed");
+  if (e != cudaSuccess) return cuda_fail(e, "output_projection launch");
+  return VMLA_OK;
 }
 
 vmla_status vmla_get_device_status(void* stream) {

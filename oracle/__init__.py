@@ -28,7 +28,10 @@ Readings where the pages are silent (each is also stated where it is used):
     (cached frames plus its own chunk, bidirectional in the chunk);
   * the query's rope part q_r,h (32 dims per head) arrives unrotated and is
     rotated with the query's own position;
-  * the softmax scale is an argument (the tests use 1/sqrt(128 + 32)).
+  * the softmax scale is an argument (the tests use 1/sqrt(128 + 32));
+  * the query, rope-query and output projections around the attention are
+    plain nn.Linear maps without bias (the pages name the Wan2.1 backbone and
+    give no formula for them): `linear`.
 
 Pins: tests/test_oracle_pins.py checks every function here against values
 the pages print (the 224 / 3072 / 92.7% cache sizes), closed forms, invariants
@@ -239,6 +242,14 @@ def chunk_attention(q_bits, q_rope_bits, w_uk_bits, w_uv_bits, cache_bits, n_kv:
                 P = _softmax_rows(scale * (Q_h @ K_h.T))
                 out[b, i0:i0 + len(sel), h] = P @ V_h
     return out
+
+
+def linear(x_bits, w_bits) -> np.ndarray:
+    """y = x . W^T in float64 for x[..., in] and an nn.Linear weight W[out, in] (bf16 bits):
+    the query, rope-query and output projections around the latent attention."""
+    x = decode_bf16(x_bits)
+    w = decode_bf16(w_bits)
+    return x @ w.T
 
 
 def materialized_kv(w_uk_bits, w_uv_bits, cache_bits, n_kv: int) -> np.ndarray:

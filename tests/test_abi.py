@@ -80,6 +80,19 @@ def test_attention_validation(vm):
     assert L.vmla_selftest_wait_timeout(10, None) == 1
 
 
+def test_projection_validation(vm):
+    L = vm.lib
+    assert L.vmla_query_projection(A, A, A, 1, 192, 1536, 12, A, None, None) == 1
+    assert L.vmla_query_projection(A, A, A + 8, 1, 192, 1536, 12, A, A, None) == 1   # misaligned
+    assert L.vmla_query_projection(A, A, A, 0, 192, 1536, 12, A, A, None) == 1       # batch
+    assert L.vmla_query_projection(A, A, A, 1, 192, 1500, 12, A, A, None) == 2       # d_model % 64
+    assert L.vmla_query_projection(A, A, A, 1, 192, 1536, 0, A, A, None) == 1        # heads
+    assert L.vmla_output_projection(A, A, 1, 192, 12, 1536, None, None) == 1
+    assert L.vmla_output_projection(A, A, 1, 0, 12, 1536, A, None) == 1              # n_tok
+    assert L.vmla_output_projection(A, A, 1, 192, 12, 1600, A, None) == 2            # d_model % 128
+    assert "d_model" in vm.vmla_last_error()
+
+
 def test_binding_rejects_non_cuda_tensors(vm):
     import torch
     x = torch.zeros(1, 4, 64, dtype=torch.bfloat16)

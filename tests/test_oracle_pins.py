@@ -396,6 +396,40 @@ def _rope_sign_flipped(v, t, r, c):
     return out
 
 
+def test_linear_hand_example_and_orientation():
+    # A non-square weight [out=3, in=5]: a transposed operand cannot even produce [2, 3].
+    x = np.array([[1, 2, 0, 0, 0], [0, 0, 0, 0, 1]], dtype=np.float32)
+    W = np.array([[1, 0, 0, 0, 0], [0, 1, 0, 0, 0], [0, 0, 0, 0, 2]], dtype=np.float32)
+    y = oracle.linear(workload.bf16_bits(x), workload.bf16_bits(W))
+    assert y.shape == (2, 3)
+    assert np.array_equal(y, np.array([[1.0, 2.0, 0.0], [0.0, 0.0, 2.0]]))
+
+
+def test_linear_identity_and_bruteforce():
+    rng = np.random.default_rng(21)
+    xb = workload.bf16_bits(rng.standard_normal((4, 6)).astype(np.float32))
+    eye = workload.bf16_bits(np.eye(6, dtype=np.float32))
+    assert np.array_equal(oracle.linear(xb, eye), oracle.decode_bf16(xb))
+    wb = workload.bf16_bits(rng.standard_normal((7, 6)).astype(np.float32))
+    xs, ws = workload.bf16_to_f32(xb).tolist(), workload.bf16_to_f32(wb).tolist()
+    y = oracle.linear(xb, wb)
+    for i in range(4):
+        for o in range(7):
+            exact = math.fsum(xs[i][k] * ws[o][k] for k in range(6))
+            assert abs(y[i, o] - exact) <= 1e-14 * (1 + abs(exact))
+
+
+def test_linear_batched_leading_dims():
+    # [B, n, D] inputs keep their leading dims; each token is projected on its own.
+    rng = np.random.default_rng(22)
+    xb = workload.bf16_bits(rng.standard_normal((2, 3, 8)).astype(np.float32))
+    wb = workload.bf16_bits(rng.standard_normal((5, 8)).astype(np.float32))
+    y = oracle.linear(xb, wb)
+    assert y.shape == (2, 3, 5)
+    for b in range(2):
+        np.testing.assert_array_equal(y[b, 1], oracle.linear(xb[b, 1:2], wb)[0])
+
+
 def test_planted_rope_sign_error_is_caught():
     rng = np.random.default_rng(16)
     v = rng.standard_normal(32)

@@ -36,6 +36,10 @@ _STREAM = {
     "w_kr": 12,
     "w_uk": 13,
     "w_uv": 14,
+    "w_q": 15,
+    "w_qr": 16,
+    "w_o": 17,
+    "o": 18,
     "k_dense": 21,
     "v_dense": 22,
 }
@@ -108,6 +112,13 @@ class Workload:
         """Dense per-head attention FLOPs (QK^T and PV, d = 128)."""
         return 2.0 * 2.0 * self.batch * self.n_q * self.heads * self.n_kv * self.d_head
 
+    def io_projection_flops(self) -> float:
+        """Query + rope-query projection (D -> H*160) and output projection (H*128 -> D)
+        of the current chunk's tokens."""
+        n = self.batch * self.n_q
+        return 2.0 * n * self.d_model * self.heads * (self.d_head + self.d_r) + \
+            2.0 * n * self.heads * self.d_head * self.d_model
+
     def append_flops(self, n_tok: int | None = None) -> float:
         n = self.n_q if n_tok is None else n_tok
         return 2.0 * self.batch * n * (self.d_c + self.d_r) * self.d_model
@@ -158,6 +169,25 @@ def layer_weights(w: Workload, layer: int = 0) -> dict:
         "w_uk": normal_bf16(s, (layer, _STREAM["w_uk"]), (H * dh, dc), std=dc ** -0.5),
         "w_uv": normal_bf16(s, (layer, _STREAM["w_uv"]), (H * dh, dc), std=dc ** -0.5),
     }
+
+
+def io_weights(w: Workload, layer: int = 0) -> dict:
+    """The projections around the attention of one layer, nn.Linear layout [out, in]:
+    w_q [H*128, D] and w_qr [H*32, D] map hidden states to content / rope queries,
+    w_o [D, H*128] maps the concatenated head outputs back to the model width."""
+    D, H, dh, dr = w.d_model, w.heads, w.d_head, w.d_r
+    s = w.seed
+    return {
+        "w_q": normal_bf16(s, (layer, _STREAM["w_q"]), (H * dh, D), std=D ** -0.5),
+        "w_qr": normal_bf16(s, (layer, _STREAM["w_qr"]), (H * dr, D), std=D ** -0.5),
+        "w_o": normal_bf16(s, (layer, _STREAM["w_o"]), (D, H * dh), std=(H * dh) ** -0.5),
+    }
+
+
+def head_outputs(w: Workload, layer: int = 0) -> np.ndarray:
+    """A stand-in attention output o [B, n_q, H, 128] ~ N(0, 1) for testing W_O alone."""
+    return np.stack([normal_bf16(w.seed + b * 7919, (layer, _STREAM["o"]), (w.n_q, w.heads, w.d_head))
+                     for b in range(w.batch)])
 
 
 def sample_activations(w: Workload, sample: int, layer: int = 0, step: int = 0) -> dict:
