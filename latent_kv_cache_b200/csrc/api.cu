@@ -249,6 +249,8 @@ vmla_status vmla_query_projection(const uint16_t* x, const uint16_t* w_q, const 
   if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "query_projection: heads must be in [1, 512]");
   if (d_model < 64 || d_model > 65536 || d_model % 64 != 0)
     return fail(VMLA_ERR_UNSUPPORTED, "query_projection: d_model must be a multiple of 64 in [64, 65536]");
+  if (((int64_t)batch * n_tok + 255) / 256 * ((heads * (vmla::kDh + vmla::kDr) + 255) / 256) > 0x7FFFFFFF)
+    return fail(VMLA_ERR_UNSUPPORTED, "query_projection: more than 2^31 - 1 output tiles");
   int* status = vmla::device_status_word();
   if (!status) return fail(VMLA_ERR_CUDA, "query_projection: no CUDA device");
   bool enc_fail = false;
@@ -269,6 +271,8 @@ vmla_status vmla_output_projection(const uint16_t* o, const uint16_t* w_o, int32
   if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "output_projection: heads must be in [1, 512]");
   if (d_model < 128 || d_model > 65536 || d_model % 128 != 0)
     return fail(VMLA_ERR_UNSUPPORTED, "output_projection: d_model must be a multiple of 128 in [128, 65536]");
+  if (((int64_t)batch * n_tok + 255) / 256 * ((d_model + 255) / 256) > 0x7FFFFFFF)
+    return fail(VMLA_ERR_UNSUPPORTED, "output_projection: more than 2^31 - 1 output tiles");
   int* status = vmla::device_status_word();
   if (!status) return fail(VMLA_ERR_CUDA, "output_projection: no CUDA device");
   bool enc_fail = false;

@@ -7,10 +7,22 @@
 //     q_r = x . W_QR^T   [tokens, H*32]   (RoPE3D is applied by the attention kernel)
 // and the output projection is the one-matrix case  y = o . W_O^T.
 //
-// One CTA = a 128 x 256 tile (N = 256 MMAs, the efficient tcgen05 shape);
-// 192 threads: warp 0 TMA producer (4-stage ring of [A 128x64 | B 256x64]
-// 128B-swizzled k blocks), warp 1 TMEM allocation + MMA issue, warps 2-5 the
-// epilogue (TMEM lane = output row).
+// Design: a persistent kernel over clusters of two CTAs on a CTA pair
+// (tcgen05 cta_group::2).  One pair computes a 256 x 256 tile: CTA r stages A rows
+// [128r, 128r + 128) and B rows [128r, 128r + 128) of the tile, and the leader
+// CTA's single MMA thread issues M = 256, N = 256 MMAs that read both CTAs' shared
+// memory and leave rows [128r, 128r + 128) of the fp32 tile in CTA r's TMEM.
+// Every CTA therefore loads (128 + 128) x 64 operands per 128 x 256 x 64 of MMA
+// work, half the bytes per FLOP of a one-CTA 128 x 256 tile; on this part the
+// one-CTA tile was bound by the L2 -> SM operand traffic.
+// TMEM holds two 256-column accumulators, so the epilogue of one tile overlaps
+// the main loop of the next.
+//
+// 192 threads per CTA: warp 0 TMA producer (6-stage ring of [A 128x64 | B 128x64]
+// 128B-swizzled k blocks), warp 1 TMEM allocation (+ the MMA issue in the leader),
+// warps 2-5 the epilogue (TMEM lane = output row).  No multicast anywhere: each
+// CTA loads its own operands and the MMA completions are committed to each CTA's
+// barrier separately.  Every wait is bounded (abort flag + device status word).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,16 +33,25 @@ namespace vmla {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kStages = 4;
-constexpr uint32_t kABytes = kBM * kBK * 2;           // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;           // 32 KB (two 128-row halves)
-constexpr uint32_t kStageBytes = kABytes + kBBytes;   // 48 KB
-constexpr uint32_t kBarOff = kStages * kStageBytes;   // 196608
+constexpr int kTileM = 256, kTileN = 256, kBK = 64;  // per CTA pair
+constexpr int kHalf = 128;                           // rows of A and of B each CTA stages
+constexpr int kStages = 6;
+constexpr uint32_t kABytes = kHalf * kBK * 2;        // 16 KB
+constexpr uint32_t kBBytes = kHalf * kBK * 2;        // 16 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;  // 32 KB
+constexpr uint32_t kBarOff = kStages * kStageBytes;  // 196608
 constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 
-enum { G_FULL0 = 0, G_EMPTY0 = kStages, G_DONE = 2 * kStages, G_DRAIN, G_COUNT };
+enum {
+  G_FULL0 = 0,                   // leader: both CTAs' operand bytes of a stage landed
+  G_EMPTY0 = kStages,            // each CTA: the MMAs reading a stage are done
+  G_ACCF0 = 2 * kStages,         // each CTA: accumulator a holds a finished tile (x2)
+  G_ACCE0 = 2 * kStages + 2,     // leader: both CTAs' epilogues drained accumulator a (x2)
+  G_DRAIN = 2 * kStages + 4,
+  G_COUNT
+};
+static_assert(8 * G_COUNT + 8 <= 256, "barrier area");
 
 struct GemmMaps {
   CUtensorMap a;   // [M, K] box (64, 128)
@@ -43,14 +64,103 @@ struct GemmParams {
   uint16_t* c1;
   int64_t ldc0, ldc1;
   int m, n0, n1, k;
+  int tiles_m, tiles_n;
   int* status;
   uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ uint32_t gbar(uint32_t base, int i) { return base + 8u * i; }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (barriers that receive the peer CTA's arrivals).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const WaitCtl& ctl, int code) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*ctl.abort_flag) return false;
+    if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      *ctl.abort_flag = 1;
+      atomicCAS(ctl.status, 0, code);
+      return false;
+    }
+  }
+}
+// 2-D tile load into this CTA's shared memory; the completed bytes are counted on
+// `bar_cluster`, which may be the leader CTA's barrier (the cta_group::2 form).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar_cluster, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+// Arrive on one CTA's barrier once this thread's earlier pair MMAs have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_bf16(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
+    k_gemm_bf16_pair(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023) & ~uintptr_t(1023)) - raw);  // kSmemBytes keeps 1 KB of slack
@@ -59,8 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * G_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int n0 = blockIdx.y * kBN;
+  const uint32_t rank = cluster_rank();  // 0 = leader (issues the MMAs)
+  const int pair = (int)cluster_id_x(), n_pairs = (int)cluster_count_x();
+  const int n_tiles = p.tiles_m * p.tiles_n;
   const int nk = p.k / kBK;
 
   if (threadIdx.x == 0) {
@@ -68,17 +179,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(gbar(bars, G_FULL0 + s), 1);
       mbar_init(gbar(bars, G_EMPTY0 + s), 1);
     }
-    mbar_init(gbar(bars, G_DONE), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(gbar(bars, G_ACCF0 + a), 1);
+      mbar_init(gbar(bars, G_ACCE0 + a), 8);  // 4 epilogue warps in each of the two CTAs
+    }
     mbar_init(gbar(bars, G_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
@@ -88,25 +202,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&maps.a);
       tma_prefetch_desc(&maps.b0);
       tma_prefetch_desc(&maps.b1);
-      int last_use[kStages] = {-1, -1, -1, -1};
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % kStages, use = kb / kStages;
-        if (use > 0 && !(ok = mbar_wait(gbar(bars, G_EMPTY0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer)))
-          break;
-        const uint32_t sa = base + st * kStageBytes, fb = gbar(bars, G_FULL0 + st);
-        mbar_arrive_expect_tx(fb, kStageBytes);
-        tma_load_2d(sa, &maps.a, fb, kb * kBK, m0);
+      int last_use[kStages];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {  // each 128-row half of the tile comes from B0 or B1
-          const int row = n0 + 128 * half;
-          const uint32_t dst = sa + kABytes + half * (kBBytes / 2);
-          if (row < p.n0) tma_load_2d(dst, &maps.b0, fb, kb * kBK, row);
-          else tma_load_2d(dst, &maps.b1, fb, kb * kBK, row - p.n0);
+      for (int s = 0; s < kStages; ++s) last_use[s] = -1;
+      int g = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
+        const int m0 = (t / p.tiles_n) * kTileM + kHalf * (int)rank;
+        const int nrow = (t % p.tiles_n) * kTileN + kHalf * (int)rank;  // this CTA's half of the N tile
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int st = g % kStages, use = g / kStages;
+          if (use > 0 && !(ok = mbar_wait(gbar(bars, G_EMPTY0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer)))
+            break;
+          const uint32_t sa = base + st * kStageBytes;
+          const uint32_t fb = map_to_rank(gbar(bars, G_FULL0 + st), 0);
+          if (rank == 0) mbar_arrive_expect_tx(gbar(bars, G_FULL0 + st), 2 * kStageBytes);
+          tma_load_2d_pair(sa, &maps.a, fb, kb * kBK, m0);
+          if (nrow < p.n0) tma_load_2d_pair(sa + kABytes, &maps.b0, fb, kb * kBK, nrow);
+          else tma_load_2d_pair(sa + kABytes, &maps.b1, fb, kb * kBK, nrow - p.n0);
+          last_use[st] = use;
         }
-        last_use[st] = use;
       }
-      if (!ok) {
+      if (!ok && rank == 0) {
+        // Give in-flight loads (counted on the leader's barriers) time to land.
         for (int s = 0; s < kStages; ++s) {
           if (last_use[s] < 0) continue;
           const uint64_t t0 = globaltimer_ns();
@@ -117,26 +235,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16_f32(kBM, kBN, false, false);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kId = idesc_bf16_f32(kTileM, kTileN, false, false);
+      const uint32_t peer = 1;
+      int g = 0, i = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        const int st = kb % kStages;
-        ok = mbar_wait(gbar(bars, G_FULL0 + st), (kb / kStages) & 1, ctl, kDevTimeoutMma);
-        if (!ok) break;
+      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++i) {
+        const int acc = i & 1, acc_use = i >> 1;
+        if (acc_use > 0 &&
+            !(ok = mbar_wait_cluster(gbar(bars, G_ACCE0 + acc), (acc_use - 1) & 1, ctl, kDevTimeoutMma)))
+          break;
         tc_fence_after();
-        const uint32_t sa = base + st * kStageBytes;
-        const uint64_t a0 = smem_desc(sa, 16, 1024, kSw128);
-        const uint64_t b0 = smem_desc(sa + kABytes, 16, 1024, kSw128);
+        const uint32_t d = tmem + (uint32_t)(acc * kTileN);
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int st = g % kStages;
+          if (!(ok = mbar_wait(gbar(bars, G_FULL0 + st), (g / kStages) & 1, ctl, kDevTimeoutMma))) break;
+          tc_fence_after();
+          const uint32_t sa = base + st * kStageBytes;
+          const uint64_t a0 = smem_desc(sa, 16, 1024, kSw128);
+          const uint64_t b0 = smem_desc(sa + kABytes, 16, 1024, kSw128);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)  // +32 bytes = +2 in the descriptor's address field
-          umma_ss(tmem, a0 + 2u * k, b0 + 2u * k, kId, (kb > 0 || k > 0) ? 1u : 0u);
-        umma_commit(gbar(bars, G_EMPTY0 + st));
+          for (int k = 0; k < kBK / 16; ++k)  // +32 bytes = +2 in the descriptor's address field
+            umma_ss_pair(d, a0 + 2u * k, b0 + 2u * k, kId, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit_pair(gbar(bars, G_EMPTY0 + st));
+          umma_commit_pair(map_to_rank(gbar(bars, G_EMPTY0 + st), peer));
+        }
+        if (!ok) break;
+        umma_commit_pair(gbar(bars, G_ACCF0 + acc));
+        umma_commit_pair(map_to_rank(gbar(bars, G_ACCF0 + acc), peer));
       }
-      if (ok) {
-        umma_commit(gbar(bars, G_DONE));
-      } else {
-        umma_commit(gbar(bars, G_DRAIN));
+      if (!ok) {
+        umma_commit_pair(gbar(bars, G_DRAIN));
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(gbar(bars, G_DRAIN), 0) && globaltimer_ns() - t0 < p.wait_limit_ns) {
         }
@@ -145,18 +274,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // Epilogue warps 2..5: TMEM lane quadrant = warp % 4, row = 32 * quadrant + lane.
     const int qd = warp & 3;
-    const int r = qd * 32 + lane;
-    const int row = m0 + r;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(gbar(bars, G_DONE), 0, ctl, kDevTimeoutSoftmax));
-    if (ok) {
+    int i = 0;
+    for (int t = pair; t < n_tiles; t += n_pairs, ++i) {
+      const int acc = i & 1, acc_use = i >> 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(gbar(bars, G_ACCF0 + acc), acc_use & 1, ctl,
+                                                        kDevTimeoutSoftmax));
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t t_row = tmem + ((uint32_t)(qd * 32) << 16);
+      const int row = (t / p.tiles_n) * kTileM + kHalf * (int)rank + qd * 32 + lane;
+      const int ncol0 = (t % p.tiles_n) * kTileN;
+      const uint32_t t_row = tmem + (uint32_t)(acc * kTileN) + ((uint32_t)(qd * 32) << 16);
       uint32_t v[32];
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < kTileN / 32; ++c) {
         tmem_ld32(t_row + 32 * c, v);
         tmem_ld_wait();
-        const int col = n0 + 32 * c;  // 32 columns never straddle N0 (a multiple of 128)
+        const int col = ncol0 + 32 * c;  // 32 columns never straddle N0 (a multiple of 128)
         if (row < p.m && col < p.n0 + p.n1) {
           uint16_t* dst = col < p.n0 ? p.c0 + (int64_t)row * p.ldc0 + col
                                      : p.c1 + (int64_t)row * p.ldc1 + (col - p.n0);
@@ -172,14 +305,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(gbar(bars, G_ACCE0 + acc), 0));  // `acc` may be reused
     }
   }
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its barriers or TMEM
   if (warp == 1) {
-    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -216,13 +352,35 @@ cudaError_t launch_gemm_pair(const uint16_t* a, const uint16_t* b0, const uint16
                              int k, uint16_t* c0, int64_t ldc0, uint16_t* c1, int64_t ldc1, int* status,
                              cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
+  static int max_pairs[64] = {0};
   *encode_failed = false;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+
+  if (!attr_done[dev]) {  // co-resident CTA pairs (one CTA per SM: shared memory and TMEM)
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, k_gemm_bf16_pair, &cfg);
+    if (e != cudaSuccess) return e;
+    max_pairs[dev] = clusters > 0 ? clusters : 1;
     attr_done[dev] = true;
   }
   GemmMaps maps;
@@ -232,9 +390,15 @@ cudaError_t launch_gemm_pair(const uint16_t* a, const uint16_t* b0, const uint16
     *encode_failed = true;
     return cudaErrorInvalidValue;
   }
-  GemmParams p{c0, n1 > 0 ? c1 : c0, ldc0, n1 > 0 ? ldc1 : ldc0, m, n0, n1, k, status, kWaitLimitNs};
-  dim3 grid((unsigned)((m + kBM - 1) / kBM), (unsigned)((n0 + n1 + kBN - 1) / kBN));
-  k_gemm_bf16<<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
+  const int tiles_m = (m + kTileM - 1) / kTileM;
+  const int tiles_n = (n0 + n1 + kTileN - 1) / kTileN;
+  GemmParams p{c0, n1 > 0 ? c1 : c0, ldc0, n1 > 0 ? ldc1 : ldc0, m, n0, n1, k, tiles_m, tiles_n, status,
+               kWaitLimitNs};
+  const int64_t tiles = (int64_t)tiles_m * tiles_n;
+  const int pairs = tiles < max_pairs[dev] ? (int)tiles : max_pairs[dev];
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_bf16_pair, maps, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
