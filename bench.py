@@ -418,6 +418,52 @@ def run_ours(args, w, rank, world, local_rank):
     }
     del kvm, out_m
 
+    # ---- latent-width sweep: append + chunk attention at d_c = 64 / 128 / 192 / 256
+    dc_sweep = {}
+    for dc in (64, 128, 192, 256):
+        wdc = wr.with_(d_c=dc)
+        wts_dc = workload.layer_weights(wdc)
+        wd_dc, wk_dc = T(wts_dc["w_dkv"]), T(wts_dc["w_kr"])
+        wuk_dc, wuv_dc = T(wts_dc["w_uk"]), T(wts_dc["w_uv"])
+        cache_dc = torch.zeros(w.batch, w.n_kv, dc + w.d_r, dtype=torch.bfloat16, device=dev)
+        x_win = T(workload.batch_activations(wdc)["x"])
+        for f0 in range(0, w.cached_frames, w.chunk_frames):
+            nf = min(w.chunk_frames, w.cached_frames - f0)
+            vm.vmla_cache_append_dc(x_win[:, f0 * per:(f0 + nf) * per].contiguous(), wd_dc, wk_dc, cache_dc,
+                                    f0 * per, f0, w.grid_h, w.grid_w)
+        del x_win
+
+        def dc_step(e=None):
+            if e is not None:
+                e[0].record(stream)
+            vm.vmla_cache_append_dc(x_chunk, wd_dc, wk_dc, cache_dc, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w,
+                                    stream)
+            if e is not None:
+                e[1].record(stream)
+            vm.vmla_chunk_attention_dc(q, qr, wuk_dc, wuv_dc, cache_dc, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w,
+                                       SCALE, out, stream)
+            if e is not None:
+                e[2].record(stream)
+
+        for _ in range(args.warmup):
+            flush_buf.zero_()
+            dc_step()
+        dc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        barrier()
+        for k in range(args.steps):
+            flush_buf.zero_()
+            dc_step(dc_ev[k])
+        barrier()
+        vm.vmla_get_device_status(stream)
+        ms_app = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in dc_ev), dist, dev) / args.steps
+        ms_att = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in dc_ev), dist, dev) / args.steps
+        dc_sweep[str(dc)] = {
+            "attention_ms": ms_att, "attention_tflops": wdc.attention_flops() / (ms_att * 1e-3) / 1e12,
+            "append_us": ms_app * 1e3, "cache_bytes_per_token": (dc + w.d_r) * 2,
+            "window_cache_mb": w.batch * w.n_kv * (dc + w.d_r) * 2 / 1e6,
+        }
+        del wd_dc, wk_dc, wuk_dc, wuv_dc, cache_dc
+
     # ---- the projections either side of the attention (same chunk, this layer's weights)
     iw = workload.io_weights(wr)
     wq, wqr, wo = T(iw["w_q"]), T(iw["w_qr"]), T(iw["w_o"])
@@ -493,6 +539,7 @@ def run_ours(args, w, rank, world, local_rank):
         "attention_layer_tokens_per_s": w.batch * w.n_q / (attn_mean * 1e-3),
         "nonabsorbed": nonabsorbed,
         "projections": projections,
+        "dc_sweep": dc_sweep,
         "dense": {"ms": dense_ms, "tflops": w.dense_flops() / (dense_ms * 1e-3) / 1e12,
                   "mla_over_dense_ms": attn_mean / dense_ms,
                   "cache_bytes_per_token": {"mla": 224 * 2, "dense": 3072 * 2}},

@@ -108,6 +108,30 @@ vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, cons
                                  uint16_t* out, void* stream);
 
 /*
+ * The same two calls for another latent width d_c (summary "Key results": batch
+ * headroom from 4.6x to at least 11.4x across latent budgets, 8.0x at the default
+ * d_c = 192; summary "Limitations": d_c = 64 loses fine detail, so d_c trades
+ * quality for efficiency).  d_c is one of 64, 128, 192, 256 (anything else returns
+ * VMLA_ERR_UNSUPPORTED); the rope key stays 32 wide, so a cached row holds
+ * d_c + 32 scalars:
+ *   w_dkv [d_c, d_model];  w_uk, w_uv [heads*128, d_c];  cache [batch, cap, d_c + 32],
+ *   row = [c (d_c) ; rotated k_r (32)].
+ * Everything else -- arguments, arithmetic order of the append (bit-exact contract),
+ * the attention's definition, limits and errors -- is as for vmla_cache_append and
+ * vmla_chunk_attention, which are these calls with d_c = 192.
+ */
+vmla_status vmla_cache_append_dc(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                                 int32_t batch, int32_t n_tok, int32_t d_model, int32_t d_c, uint16_t* cache,
+                                 int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
+                                 int32_t grid_w, void* stream);
+
+vmla_status vmla_chunk_attention_dc(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                    const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                    int32_t n_q, int32_t heads, int32_t d_c, int64_t cap, int64_t n_kv,
+                                    int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
+                                    uint16_t* out, void* stream);
+
+/*
  * vmla_dense_attention -- the per-head (3072-scalar) baseline layout, for comparison.
  * (summary "Key results": Self-Forcing's dense per-head KV cache, 3072 scalars/token.)
  *

@@ -61,6 +61,10 @@ def _load():
     lib.vmla_chunk_attention_nonabsorbed.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32,
                                                      P, i64, P, P]
     lib.vmla_chunk_attention_nonabsorbed.restype = ctypes.c_int
+    lib.vmla_cache_append_dc.argtypes = [P, P, P, i32, i32, i32, i32, P, i64, i64, i64, i32, i32, P]
+    lib.vmla_cache_append_dc.restype = ctypes.c_int
+    lib.vmla_chunk_attention_dc.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64, i64, i64, i32, i32, f32, P, P]
+    lib.vmla_chunk_attention_dc.restype = ctypes.c_int
     lib.vmla_query_projection.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P]
     lib.vmla_query_projection.restype = ctypes.c_int
     lib.vmla_output_projection.argtypes = [P, P, i32, i32, i32, i32, P, P]
@@ -133,6 +137,39 @@ def vmla_chunk_attention(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0: int, grid_
                                     _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, Nq, H, cache.shape[1],
                                     int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
                                     _ptr(out, "out"), _stream(stream)))
+
+
+def vmla_cache_append_dc(x, w_dkv, w_kr, cache, slot0: int, t0: int, grid_h: int, grid_w: int,
+                         stream=None) -> None:
+    """vmla_cache_append for latent width d_c = w_dkv.shape[0] (64, 128, 192 or 256):
+    w_dkv [d_c, D], cache [B, cap, d_c + 32]."""
+    B, n_tok, D = x.shape
+    d_c = w_dkv.shape[0]
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != d_c + D_R:
+        raise ValueError("cache must be [B, cap, d_c + 32]")
+    if w_dkv.shape[1] != D or tuple(w_kr.shape) != (D_R, D):
+        raise ValueError("w_dkv must be [d_c, D] and w_kr [32, D]")
+    _check(lib.vmla_cache_append_dc(_ptr(x, "x"), _ptr(w_dkv, "w_dkv"), _ptr(w_kr, "w_kr"), B, n_tok, D, d_c,
+                                    _ptr(cache, "cache"), cache.shape[1], int(slot0), int(t0),
+                                    int(grid_h), int(grid_w), _stream(stream)))
+
+
+def vmla_chunk_attention_dc(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0: int, grid_h: int, grid_w: int,
+                            scale: float, out, stream=None) -> None:
+    """vmla_chunk_attention for latent width d_c = w_uk.shape[1]: w_uk/w_uv [H*128, d_c],
+    cache [B, cap, d_c + 32]."""
+    B, Nq, H, dh = q.shape
+    d_c = w_uk.shape[1]
+    if dh != D_HEAD or tuple(q_rope.shape) != (B, Nq, H, D_R) or tuple(out.shape) != (B, Nq, H, D_HEAD):
+        raise ValueError("q/q_rope/out shapes do not match [B, Nq, H, 128|32]")
+    if tuple(w_uk.shape) != (H * D_HEAD, d_c) or tuple(w_uv.shape) != (H * D_HEAD, d_c):
+        raise ValueError("w_uk / w_uv must be [H*128, d_c]")
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != d_c + D_R:
+        raise ValueError("cache must be [B, cap, d_c + 32]")
+    _check(lib.vmla_chunk_attention_dc(_ptr(q, "q"), _ptr(q_rope, "q_rope"), _ptr(w_uk, "w_uk"),
+                                       _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, Nq, H, d_c, cache.shape[1],
+                                       int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
+                                       _ptr(out, "out"), _stream(stream)))
 
 
 def vmla_dense_attention(q, k, v, scale: float, out, stream=None) -> None:

@@ -10,11 +10,11 @@
 
 namespace vmla {
 cudaError_t launch_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
-                                int batch, int n_tok, int d_model, uint16_t* cache, int64_t cap,
+                                int batch, int n_tok, int d_model, int d_c, uint16_t* cache, int64_t cap,
                                 int64_t slot0, int64_t t0, int grid_h, int grid_w, cudaStream_t stream);
 cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
                                    const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
-                                   int heads, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
+                                   int heads, int d_c, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
                                    int grid_w, float scale, uint16_t* out, int* status,
                                    cudaStream_t stream, bool* encode_failed);
 cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int batch,
@@ -85,10 +85,13 @@ const char* vmla_status_string(int status) {
 
 const char* vmla_last_error(void) { return g_last_error; }
 
-vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
-                              int32_t batch, int32_t n_tok, int32_t d_model, uint16_t* cache,
-                              int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
-                              int32_t grid_w, void* stream) {
+static bool supported_dc(int32_t d_c) { return d_c == 64 || d_c == 128 || d_c == 192 || d_c == 256; }
+
+vmla_status vmla_cache_append_dc(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                                 int32_t batch, int32_t n_tok, int32_t d_model, int32_t d_c, uint16_t* cache,
+                                 int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
+                                 int32_t grid_w, void* stream) {
+  if (!supported_dc(d_c)) return fail(VMLA_ERR_UNSUPPORTED, "cache_append: d_c must be 64, 128, 192 or 256");
   if (!aligned16(x) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(cache))
     return fail(VMLA_ERR_INVALID_ARG, "cache_append: pointers must be non-null and 16-byte aligned");
   if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "cache_append: batch must be in [1, 65535]");
@@ -99,17 +102,26 @@ vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const ui
   if (slot0 < 0 || slot0 >= cap) return fail(VMLA_ERR_INVALID_ARG, "cache_append: need 0 <= slot0 < cap");
   vmla_status st = check_positions(n_tok, t0, grid_h, grid_w);
   if (st != VMLA_OK) return st;
-  cudaError_t e = vmla::launch_cache_append(x, w_dkv, w_kr, batch, n_tok, d_model, cache, cap, slot0,
+  cudaError_t e = vmla::launch_cache_append(x, w_dkv, w_kr, batch, n_tok, d_model, d_c, cache, cap, slot0,
                                             t0, grid_h, grid_w, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cache_append launch");
   return VMLA_OK;
 }
 
-vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
-                                 const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
-                                 int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv,
-                                 int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
-                                 uint16_t* out, void* stream) {
+vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                              int32_t batch, int32_t n_tok, int32_t d_model, uint16_t* cache,
+                              int64_t cap, int64_t slot0, int64_t t0, int32_t grid_h,
+                              int32_t grid_w, void* stream) {
+  return vmla_cache_append_dc(x, w_dkv, w_kr, batch, n_tok, d_model, vmla::kDc, cache, cap, slot0, t0, grid_h,
+                              grid_w, stream);
+}
+
+vmla_status vmla_chunk_attention_dc(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                    const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                    int32_t n_q, int32_t heads, int32_t d_c, int64_t cap, int64_t n_kv,
+                                    int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
+                                    uint16_t* out, void* stream) {
+  if (!supported_dc(d_c)) return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: d_c must be 64, 128, 192 or 256");
   if (!aligned16(q) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(w_uv) ||
       !aligned16(cache) || !aligned16(out))
     return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: pointers must be non-null and 16-byte aligned");
@@ -127,12 +139,21 @@ vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, cons
   int* status = vmla::device_status_word();
   if (!status) return fail(VMLA_ERR_CUDA, "chunk_attention: no CUDA device");
   bool enc_fail = false;
-  cudaError_t e = vmla::launch_chunk_attention(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap,
+  cudaError_t e = vmla::launch_chunk_attention(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, d_c, cap,
                                                n_kv, t0, grid_h, grid_w, scale, out, status,
                                                static_cast<cudaStream_t>(stream), &enc_fail);
   if (enc_fail) return fail(VMLA_ERR_CUDA, "chunk_attention: tensor-map encoding failed");
   if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
   return VMLA_OK;
+}
+
+vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                 const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
+                                 int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv,
+                                 int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
+                                 uint16_t* out, void* stream) {
+  return vmla_chunk_attention_dc(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, vmla::kDc, cap, n_kv, t0,
+                                 grid_h, grid_w, scale, out, stream);
 }
 
 vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,

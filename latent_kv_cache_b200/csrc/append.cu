@@ -2,7 +2,9 @@
 //
 // VideoMLA ("Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video
 // Diffusion", abstract and summary "Approach"): each cached token stores a
-// head-shared content latent (192) and a head-shared decoupled 3D-RoPE key (32).
+// head-shared content latent (d_c = 192 in the paper's model; the kernel is a
+// template over d_c in {64, 128, 192, 256}) and a head-shared decoupled 3D-RoPE
+// key (32).
 //
 // The arithmetic order is fixed so the result is reproducible bit for bit:
 // every output is one fp32 accumulator updated for k = 0, 1, ..., d_model-1
@@ -12,9 +14,10 @@
 // then rounded to bf16 (nearest even).  This is CUDA-core work: the tensor
 // cores do not specify their accumulation order.
 //
-// Tiling: a CTA owns 32 tokens x all 224 outputs; each of its 4 warps owns 8
-// tokens, and lane l owns outputs l + 32 i (i = 0..6), so the rope dims (outputs
-// 192..223) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
+// Tiling: a CTA owns 32 tokens (16 at d_c = 256, to stay within the register
+// budget) x all d_c + 32 outputs; each of its 4 warps owns a quarter of the
+// tokens, and lane l owns outputs l + 32 i, so the rope dims (the last 32
+// outputs) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
 // Operands are staged per 64-wide k chunk in shared memory as fp32, double
 // buffered: the global loads of chunk c+1 are issued into registers before the
 // FMAs of chunk c, and land in the other buffer after them, so their latency
@@ -27,16 +30,23 @@
 namespace vmla {
 
 namespace {
-constexpr int kTok = 32;         // tokens per CTA
 constexpr int kKc = 64;          // k chunk
 constexpr int kThreads = 128;    // 4 warps
-constexpr int kTokPerWarp = 8;
-constexpr int kOutPerLane = 7;   // 224 / 32
 constexpr int kStride = kKc + 4; // fp32 row stride in shared memory (conflict-free float4 reads)
-constexpr int kBufFloats = (kDrow + kTok) * kStride;
-constexpr int kSmemBytes = 2 * kBufFloats * 4;
-constexpr int kWVec = kDrow * 8 / kThreads;  // 16-byte W vectors per thread per chunk (14)
-constexpr int kXVec = kTok * 8 / kThreads;   // 16-byte x vectors per thread per chunk (2)
+
+template <int kDcT>
+struct AppendCfg {
+  static constexpr int kRow = kDcT + kDr;                    // cached scalars per token
+  static constexpr int kTokPerWarp = kDcT > 192 ? 4 : 8;
+  static constexpr int kTok = 4 * kTokPerWarp;               // tokens per CTA
+  static constexpr int kOutPerLane = kRow / 32;              // 3, 5, 7, 9
+  static constexpr int kBufFloats = (kRow + kTok) * kStride;
+  static constexpr int kSmemBytes = 2 * kBufFloats * 4;
+  static constexpr int kWVec = kRow * 8 / kThreads;          // 16-byte W vectors per thread per chunk
+  static constexpr int kXVec = kTok * 8 / kThreads;          // 16-byte x vectors per thread per chunk
+  static_assert(kRow % 32 == 0 && (kRow * 8) % kThreads == 0 && (kTok * 8) % kThreads == 0, "tiling");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
 
 struct AppendParams {
   const uint16_t* x;
@@ -56,11 +66,13 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float4& lo, float4
   hi = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
 }
 
+template <int kDcT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_cache_append(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
+  using A = AppendCfg<kDcT>;
+  constexpr int kDrow = A::kRow, kTok = A::kTok, kTokPerWarp = A::kTokPerWarp, kOutPerLane = A::kOutPerLane;
+  constexpr int kBufFloats = A::kBufFloats, kWVec = A::kWVec, kXVec = A::kXVec;
   extern __shared__ __align__(16) float smem_f[];
-  float* ws = smem_f;                   // [224][kStride]  weights of the chunk
-  float* xs = smem_f + kDrow * kStride; // [32][kStride]   tokens of the chunk
   const int b = blockIdx.y;
   const int tok0 = blockIdx.x * kTok;
   const int warp = threadIdx.x >> 5;
@@ -80,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; n < kWVec; ++n) {
       const int v = threadIdx.x + kThreads * n;
       const int row = v >> 3, kk = (v & 7) * 8;
-      const uint16_t* src = row < kDc ? p.w_dkv + (int64_t)row * p.d_model
-                                      : p.w_kr + (int64_t)(row - kDc) * p.d_model;
+      const uint16_t* src = row < kDcT ? p.w_dkv + (int64_t)row * p.d_model
+                                       : p.w_kr + (int64_t)(row - kDcT) * p.d_model;
       wreg[n] = __ldg(reinterpret_cast<const uint4*>(src + k0 + kk));
     }
 #pragma unroll
@@ -148,14 +160,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  // 3D rotary embedding of the rope dims (output 192 + lane).
+  // 3D rotary embedding of the rope dims (output d_c + lane, the lane's last output).
   const int pair = lane >> 1;
   const bool even = (lane & 1) == 0;
   const int per_frame = p.grid_h * p.grid_w;
 #pragma unroll
   for (int t = 0; t < kTokPerWarp; ++t) {
     const int tok = tok0 + warp * kTokPerWarp + t;
-    const float v = acc[t][6];
+    const float v = acc[t][kOutPerLane - 1];
     const float other = __shfl_xor_sync(0xffffffffu, v, 1);
     if (tok < p.n_tok) {
       const int f = tok / per_frame;
@@ -168,12 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       else cs = tab.w[col][pair - kPairsT - kPairsH];
       const float a = even ? v : other;
       const float bb = even ? other : v;
-      acc[t][6] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
-                       : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
+      acc[t][kOutPerLane - 1] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
+                                     : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
     }
   }
 
-  // Stage the 32 x 224 bf16 rows in shared memory, then write 16-byte vectors.
+  // Stage the kTok x (d_c + 32) bf16 rows in shared memory, then write 16-byte vectors.
   __syncthreads();
   __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_f);
 #pragma unroll
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kOutPerLane; ++i)
       os[(warp * kTokPerWarp + t) * kDrow + lane + 32 * i] = __float2bfloat16_rn(acc[t][i]);
   __syncthreads();
-  constexpr int kVecPerRow = kDrow * 2 / 16;  // 28
+  constexpr int kVecPerRow = kDrow * 2 / 16;
   for (int v = threadIdx.x; v < kTok * kVecPerRow; v += kThreads) {
     const int t = v / kVecPerRow, c = v - t * kVecPerRow;
     const int tok = tok0 + t;
@@ -193,28 +205,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 }
-}  // namespace
 
-cudaError_t launch_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
-                                int batch, int n_tok, int d_model, uint16_t* cache, int64_t cap,
-                                int64_t slot0, int64_t t0, int grid_h, int grid_w,
-                                cudaStream_t stream) {
+template <int kDcT>
+cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, cudaStream_t stream) {
+  using A = AppendCfg<kDcT>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_cache_append, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(k_cache_append<kDcT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         A::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  AppendParams p{x, w_dkv, w_kr, cache, cap, slot0, n_tok, d_model, grid_h, grid_w};
   static thread_local RopeTable tab;
-  const int per_frame = grid_h * grid_w;
-  build_rope_table(&tab, t0, (n_tok + per_frame - 1) / per_frame, grid_h, grid_w);
-  dim3 grid((n_tok + kTok - 1) / kTok, batch);
-  k_cache_append<<<grid, kThreads, kSmemBytes, stream>>>(p, tab);
+  const int per_frame = p.grid_h * p.grid_w;
+  build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
+  dim3 grid((p.n_tok + A::kTok - 1) / A::kTok, batch);
+  k_cache_append<kDcT><<<grid, kThreads, A::kSmemBytes, stream>>>(p, tab);
   return cudaGetLastError();
+}
+}  // namespace
+
+// d_c in {64, 128, 192, 256}; the caller has validated it.
+cudaError_t launch_cache_append(const uint16_t* x, const uint16_t* w_dkv, const uint16_t* w_kr,
+                                int batch, int n_tok, int d_model, int d_c, uint16_t* cache, int64_t cap,
+                                int64_t slot0, int64_t t0, int grid_h, int grid_w,
+                                cudaStream_t stream) {
+  AppendParams p{x, w_dkv, w_kr, cache, cap, slot0, n_tok, d_model, grid_h, grid_w};
+  switch (d_c) {
+    case 64: return launch_cache_append_t<64>(p, batch, t0, stream);
+    case 128: return launch_cache_append_t<128>(p, batch, t0, stream);
+    case 192: return launch_cache_append_t<192>(p, batch, t0, stream);
+    case 256: return launch_cache_append_t<256>(p, batch, t0, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace vmla

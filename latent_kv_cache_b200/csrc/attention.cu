@@ -17,23 +17,18 @@
 //   warps 2..9  two softmax warpgroups; a thread owns one query row (= TMEM
 //               lane) and one half of the columns of every score tile.
 //
-// Shared-memory bandwidth is the budget that sizes this design: the tensor
-// core reads its shared-memory operands and TMA writes the next key tiles
-// through the same ~128 B/clk per SM.  The query operand therefore lives in
-// tensor memory (A operand from TMEM) and only the key tiles come from shared
-// memory: per 96-key MLA tile the tensor core reads 43 KB (K) + 36 KB (V) and
-// TMA writes 43 KB, ~98 B per tensor-core cycle.
-//
+// The latent kernel is a template over the content width d_c (64, 128, 192 or
+// 256; the rope key stays 32 wide).  Its query operand Qa = [q_abs ; RoPE(q_r)]
+// (128 x (d_c + 32) bf16) sits in shared memory, laid out like a key tile.
 // MLA tensor memory (512 columns x 128 lanes, fp32 cells):
-//   [0,192)   O_lat accumulator (the prologue's q_abs lands here first)
-//   [192,288) S buffer 0 (P, bf16, overwrites its first 48 columns)
-//   [288,384) S buffer 1
-//   [384,496) Qa = [q_abs (96 cells of bf16 pairs) ; rotated q_r (16 cells)]
-//   epilogue: normalised O_lat (bf16) at [192,288), out accumulator at [288,416).
-// Per key tile j the MMA thread issues S_j = Qa K_j^T (14 MMAs, K = 16 each,
-// the last two over the 64-byte-swizzled rope block) and then O += P_{j-1}
-// C_{j-1} (6 MMAs, P read from TMEM, C read MN-major from the same shared-memory
-// tile that served as K: keys and values are one tile).
+//   [0, d_c)    O_lat accumulator (the prologue's q_abs lands here first)
+//   [256, 384)  S buffer 0 (P, bf16, overwrites its first 64 cells)
+//   [384, 512)  S buffer 1
+//   epilogue: normalised O_lat (bf16, d_c/2 cells) at 256, out accumulator at 384.
+// Per 128-key tile j the MMA thread issues S_j = Qa K_j^T (d_c/16 + 2 MMAs,
+// K = 16 each, the last two over the 64-byte-swizzled rope block) and then
+// O += P_{j-1} C_{j-1} (8 MMAs of N = d_c, P read from TMEM, C read MN-major from
+// the same shared-memory tile that served as K: keys and values are one tile).
 // The softmax keeps the running max in log2 units and rescales O only when the
 // max grows by more than 8 (P stays <= 2^8 in bf16).
 #include <cuda.h>
@@ -57,28 +52,31 @@ constexpr uint32_t kTmemCols = 512;
 // [B, n_kv, 2H, 128] buffer, the rope key straight from the latent cache).
 enum Kind : int { kKindMla = 0, kKindDense = 1, kKindMat = 2 };
 
-// Per-variant configuration.
-template <int kKind>
+// Per-variant configuration (kDcT: content width of the latent variant).
+template <int kKind, int kDcT = kDc>
 struct Cfg;
 
-// MLA: the Qa operand (128 x 224 bf16) sits in shared memory (SS MMAs for the
-// scores): O (192) + two 128-key S buffers (256) + Qa (112) would exceed the
-// 512 TMEM columns, and 128-key score tiles matter more than the A source
+// MLA: the Qa operand (128 x (d_c + 32) bf16) sits in shared memory (SS MMAs for
+// the scores): O (d_c) + two 128-key S buffers (256) + Qa in TMEM would exceed
+// the 512 TMEM columns, and 128-key score tiles matter more than the A source
 // (a K = 16 tcgen05.mma takes at least ~93 cycles, so narrower N loses).
-template <>
-struct Cfg<kKindMla> {
-  static constexpr int kBN = 128;                              // keys per tile
-  static constexpr int kStages = 3;
-  static constexpr uint32_t kBlkRows = 128 * 128;              // one 128B-swizzled block of a key tile
-  static constexpr uint32_t kStage = 3 * kBlkRows + 128 * 64;  // [c: 3 blocks | k_r: 128 x 64 B] = 57344
-  static constexpr uint32_t kQaBytes = kStage;                 // Qa tile, same block structure
-  static constexpr int kOCols = kDc;
+// The ring is as deep as shared memory allows: 6, 4, 3, 2 stages.
+template <int kDcT>
+struct Cfg<kKindMla, kDcT> {
+  static_assert(kDcT == 64 || kDcT == 128 || kDcT == 192 || kDcT == 256, "d_c");
+  static constexpr int kNb = kDcT / 64;                          // 128B-swizzled content blocks
+  static constexpr int kBN = 128;                                // keys per tile
+  static constexpr int kStages = kDcT == 64 ? 6 : kDcT == 128 ? 4 : kDcT == 192 ? 3 : 2;
+  static constexpr uint32_t kBlkRows = 128 * 128;                // one 128B-swizzled block of a key tile
+  static constexpr uint32_t kStage = kNb * kBlkRows + 128 * 64;  // [c: kNb blocks | k_r: 128 x 64 B]
+  static constexpr uint32_t kQaBytes = kStage;                   // Qa tile, same block structure
+  static constexpr int kOCols = kDcT;
   static constexpr uint32_t kTmemS0 = 256, kTmemS1 = 384;
 };
 
 // Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
-template <>
-struct Cfg<kKindDense> {
+template <int kDcT>
+struct Cfg<kKindDense, kDcT> {
   static constexpr int kBN = 128;
   static constexpr int kStages = 3;
   static constexpr uint32_t kBlkRows = 128 * 128;
@@ -90,8 +88,8 @@ struct Cfg<kKindDense> {
 
 // Materialised keys/values: Q = [q_h ; RoPE(q_r)] (80 cells) in TMEM; key tile =
 // [content 128 ; rope 32], value tile 128.
-template <>
-struct Cfg<kKindMat> {
+template <int kDcT>
+struct Cfg<kKindMat, kDcT> {
   static constexpr int kBN = 128;
   static constexpr int kStages = 3;
   static constexpr uint32_t kBlkRows = 128 * 128;
@@ -104,22 +102,27 @@ struct Cfg<kKindMat> {
 constexpr uint32_t kBlk128 = 128 * 128;  // 128 rows x 128 B: prologue / epilogue operand blocks
 constexpr uint32_t kTmemO = 0;
 
-template <int kKind>
+template <int kKind, int kDcT = kDc>
 struct Layout {
-  static constexpr uint32_t kRingOff = Cfg<kKind>::kQaBytes;
-  static constexpr uint32_t kBarOff = kRingOff + Cfg<kKind>::kStages * Cfg<kKind>::kStage;
+  using C = Cfg<kKind, kDcT>;
+  static constexpr uint32_t kRingOff = C::kQaBytes;
+  static constexpr uint32_t kBarOff = kRingOff + C::kStages * C::kStage;
   static constexpr uint32_t kRedOff = kBarOff + 512;
   static constexpr uint32_t kUsed = kRedOff + 2 * 2 * 128 * 4;
   static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
   static constexpr uint32_t kMaxPad = kBytes - kUsed;  // alignment slack the kernel checks for
+  static_assert(kUsed + 512 <= 232448, "shared memory (with at least 512 B of alignment slack)");
+  static_assert(C::kStages <= 8, "barrier slots");
 };
-static_assert(Layout<kKindMla>::kBytes <= 232448 && Layout<kKindDense>::kBytes <= 232448 &&
-              Layout<kKindMat>::kBytes <= 232448, "shared memory");
-static_assert(Layout<kKindMla>::kMaxPad >= 512 && Layout<kKindDense>::kMaxPad >= 512 &&
-              Layout<kKindMat>::kMaxPad >= 512, "alignment slack");
-// The MLA prologue parks q (2 blocks) and W_UK (3 blocks) in the first ring stages.
-static_assert(5 * kBlk128 <= 2 * Cfg<kKindMla>::kStage, "prologue operands fit in stages 0-1");
-static_assert(2 * kBlk128 <= Cfg<kKindMla>::kStage && kBlk128 <= Cfg<kKindMla>::kStage, "W_UV blocks fit");
+// The MLA prologue parks q (2 blocks) and W_UK_h (d_c/64 blocks) in ring stages
+// 0-1; the epilogue's W_UV_h (d_c/64 blocks) is one ring item.
+template <int kDcT>
+constexpr bool mla_fits() {
+  using C = Cfg<kKindMla, kDcT>;
+  return (2 + C::kNb) * kBlk128 <= 2 * C::kStage && C::kNb * kBlk128 <= C::kStage && C::kStages >= 2 &&
+         kDcT + 256 <= (int)kTmemCols && kDcT / 2 <= 128;
+}
+static_assert(mla_fits<64>() && mla_fits<128>() && mla_fits<192>() && mla_fits<256>(), "MLA layout");
 
 enum Bar {
   B_PRO = 0, B_QABS, B_QA,
@@ -230,11 +233,11 @@ __device__ __forceinline__ bool exchange(const SoftmaxThread& t, uint32_t bars, 
 }
 
 // Softmax step for key tile j.  Returns false on abort.
-template <int kKind>
+template <int kKind, int kDcT>
 __device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const SoftmaxThread& t,
                                              const AttnParams& p, const WaitCtl& ctl,
                                              float& m_run, float& l_part) {
-  using C = Cfg<kKind>;
+  using C = Cfg<kKind, kDcT>;
   constexpr int kW = C::kBN / 2;  // score columns per thread (48 or 64)
   const int sb = j & 1;
   if (!warp_wait(bar_addr(bars, B_SF0 + sb), (j >> 1) & 1, ctl)) return false;
@@ -357,14 +360,15 @@ __device__ __forceinline__ void rope_query(const AttnParams& p, const RopeTable*
 
 // ---------------------------------------------------------------------------
 // The attention kernel.  kMla: latent chunk attention (absorbed W_UK, [c ; k_r]
-// tiles, W_UV epilogue); otherwise the dense per-head baseline (d = 128).
+// tiles, W_UV epilogue) with content width kDcT; kMat: attention over
+// materialised per-head keys/values; otherwise the dense per-head baseline.
 // ---------------------------------------------------------------------------
-template <int kKind, class Maps>
+template <int kKind, int kDcT, class Maps>
 __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p, const RopeTable* tab) {
   constexpr bool kMla = kKind == kKindMla;
   constexpr bool kMat = kKind == kKindMat;
-  using C = Cfg<kKind>;
-  using L = Layout<kKind>;
+  using C = Cfg<kKind, kDcT>;
+  using L = Layout<kKind, kDcT>;
   constexpr int kBN = C::kBN;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kStage = C::kStage;
@@ -376,7 +380,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     return;
   }
   uint8_t* smem = smem_raw + pad;
-  const uint32_t qa = smem_u32(smem);    // MLA: Qa tile (3 SW128 blocks + SW64 rope block)
+  const uint32_t qa = smem_u32(smem);    // MLA: Qa tile (d_c/64 SW128 blocks + SW64 rope block)
   const uint32_t st0 = qa + L::kRingOff; // ring stage s at st0 + s * kStage
   const uint32_t bars = qa + L::kBarOff;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * B_COUNT);
@@ -433,20 +437,20 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         tma_prefetch_desc(&maps.wuv);
         tma_prefetch_desc(&maps.c);
         tma_prefetch_desc(&maps.kr);
-        // Prologue operands borrow ring stages 0-1: q tile (2 blocks) then W_UK_h (3 blocks).
-        mbar_arrive_expect_tx(bar_addr(bars, B_PRO), 5 * kBlk128);
+        // Prologue operands borrow ring stages 0-1: q tile (2 blocks) then W_UK_h (d_c/64 blocks).
+        mbar_arrive_expect_tx(bar_addr(bars, B_PRO), (2 + C::kNb) * kBlk128);
         tma_load_4d(st0, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
         tma_load_4d(st0 + kBlk128, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
-        tma_load_2d(st0 + 2 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 0, h * kDh);
-        tma_load_2d(st0 + 3 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 64, h * kDh);
-        tma_load_2d(st0 + 4 * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 128, h * kDh);
+#pragma unroll
+        for (int i = 0; i < C::kNb; ++i)
+          tma_load_2d(st0 + (2 + i) * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 64 * i, h * kDh);
       } else {
         tma_prefetch_desc(&maps.k);
         tma_prefetch_desc(&maps.v);
         if constexpr (kMat) tma_prefetch_desc(&maps.kr);
       }
-      // MLA: n_tiles key tiles, then W_UV_h blocks {0,1} and {2} as two more ring items.
-      const int n_items = kMla ? n_tiles + 2 : n_tiles;
+      // MLA: n_tiles key tiles, then the W_UV_h blocks as one more ring item.
+      const int n_items = kMla ? n_tiles + 1 : n_tiles;
       for (int i = 0; i < n_items; ++i) {
         const int st = i % kStages, use = i / kStages;
         const uint32_t sa = st0 + st * kStage;
@@ -461,17 +465,13 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         if constexpr (kMla) {
           if (i < n_tiles) {
             mbar_arrive_expect_tx(fb, kStage);
-            tma_load_3d(sa, &maps.c, fb, 0, kv0, b);
-            tma_load_3d(sa + C::kBlkRows, &maps.c, fb, 64, kv0, b);
-            tma_load_3d(sa + 2 * C::kBlkRows, &maps.c, fb, 128, kv0, b);
-            tma_load_3d(sa + 3 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
-          } else if (i == n_tiles) {
-            mbar_arrive_expect_tx(fb, 2 * kBlk128);
-            tma_load_2d(sa, &maps.wuv, fb, 0, h * kDh);
-            tma_load_2d(sa + kBlk128, &maps.wuv, fb, 64, h * kDh);
+#pragma unroll
+            for (int blk = 0; blk < C::kNb; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
+            tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
           } else {
-            mbar_arrive_expect_tx(fb, kBlk128);
-            tma_load_2d(sa, &maps.wuv, fb, 128, h * kDh);
+            mbar_arrive_expect_tx(fb, C::kNb * kBlk128);
+#pragma unroll
+            for (int blk = 0; blk < C::kNb; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
           }
         } else {
           const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
@@ -501,9 +501,9 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       if constexpr (kMla) {
         ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
         if (ok) {
-          constexpr uint32_t kIdQabs = idesc_bf16_f32(128, kDc, false, true);
+          constexpr uint32_t kIdQabs = idesc_bf16_f32(128, kDcT, false, true);
           tc_fence_after();
-          // q_abs = q_h . W_UK_h (M 128, N 192, K 128): q K-major, W_UK MN-major.
+          // q_abs = q_h . W_UK_h (M 128, N d_c, K 128): q K-major, W_UK MN-major.
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
@@ -538,13 +538,15 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         const uint32_t sa = st0 + st * kStage;
         const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
         if constexpr (kMla) {
-          // S = Qa . [c ; k_r]^T (K = 224): 12 steps over the 128B-swizzled content
-          // blocks, 2 over the 64B-swizzled rope block; Qa and the key tile share offsets.
+          // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
+          // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
+          // share offsets.
+          constexpr int kCs = 4 * C::kNb;
 #pragma unroll
-          for (int k = 0; k < 14; ++k) {
-            const uint32_t off = k < 12 ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : 3 * C::kBlkRows + (k - 12) * 32;
-            const uint32_t sbo = k < 12 ? 1024 : 512;
-            const uint32_t lay = k < 12 ? kSw128 : kSw64;
+          for (int k = 0; k < kCs + 2; ++k) {
+            const uint32_t off = k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32;
+            const uint32_t sbo = k < kCs ? 1024 : 512;
+            const uint32_t lay = k < kCs ? kSw128 : kSw64;
             umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
           }
         } else {
@@ -565,17 +567,16 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       if constexpr (kMla) {
         if (ok) {
           constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
-          const int s01 = n_tiles % kStages, s2 = (n_tiles + 1) % kStages;
-          ok = mbar_wait(bar_addr(bars, B_KVF0 + s01), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
-               mbar_wait(bar_addr(bars, B_KVF0 + s2), ((n_tiles + 1) / kStages) & 1, ctl, kDevTimeoutMma) &&
+          const int sw = n_tiles % kStages;
+          ok = mbar_wait(bar_addr(bars, B_KVF0 + sw), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
                mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
           if (ok) {
             tc_fence_after();
-            const uint32_t wb[3] = {st0 + s01 * kStage, st0 + s01 * kStage + kBlk128, st0 + s2 * kStage};
-            // out = O_lat/l . W_UV_h^T (M 128, N 128, K 192): A from TMEM, W_UV K-major.
+            const uint32_t wb = st0 + sw * kStage;
+            // out = O_lat/l . W_UV_h^T (M 128, N 128, K d_c): A from TMEM, W_UV K-major.
 #pragma unroll
-            for (int k = 0; k < 12; ++k) {
-              const uint64_t bd = smem_desc(wb[k >> 2] + (k & 3) * 32, 16, 1024, kSw128);
+            for (int k = 0; k < kDcT / 16; ++k) {
+              const uint64_t bd = smem_desc(wb + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
               umma_ts(tmem + C::kTmemS1, tmem + C::kTmemS0 + k * 8, bd, kIdOut, k > 0);
             }
             umma_commit(bar_addr(bars, B_OUT));
@@ -601,11 +602,12 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       ok = warp_wait(bar_addr(bars, B_QABS), 0, ctl);
       if (ok) {
         tc_fence_after();
-        // q_abs (fp32, TMEM) -> bf16 Qa tile in shared memory; this half: columns [96 half, +96).
+        // q_abs (fp32, TMEM) -> bf16 Qa tile in shared memory; this half: columns
+        // [d_c/2 half, +d_c/2).
         uint32_t v[32];
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          const int col = 96 * t.half + 32 * c;
+        for (int c = 0; c < C::kNb; ++c) {
+          const int col = (kDcT / 2) * t.half + 32 * c;
           tmem_ld32(t.t_row + kTmemO + col, v);
           tmem_ld_wait();
 #pragma unroll
@@ -622,7 +624,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             w.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
             w.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
             w.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
-            st_sw64_chunk(smem + 3 * C::kBlkRows, t.r, c, w);
+            st_sw64_chunk(smem + C::kNb * C::kBlkRows, t.r, c, w);
           }
         }
         fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
@@ -659,7 +661,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       mbar_arrive(bar_addr(bars, B_QA));
     }
     float m_run = -INFINITY, l_part = 0.0f;
-    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kKind>(j, bars, t, p, ctl, m_run, l_part);
+    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kKind, kDcT>(j, bars, t, p, ctl, m_run, l_part);
     float l_other = 0.0f;
     if (ok) ok = exchange(t, bars, n_tiles, l_part, l_other, ctl);
     if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
@@ -669,15 +671,16 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
       uint32_t v[32];
       if constexpr (kMla) {
-        // Normalised O_lat -> bf16 A operand of the W_UV MMA (this half: latent [96 half, +96)).
+        // Normalised O_lat -> bf16 A operand of the W_UV MMA (this half: latent
+        // [d_c/2 half, +d_c/2), i.e. d_c/4 cells).
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          tmem_ld32(t.t_row + kTmemO + 96 * t.half + 32 * c, v);
+        for (int c = 0; c < C::kNb; ++c) {
+          tmem_ld32(t.t_row + kTmemO + (kDcT / 2) * t.half + 32 * c, v);
           tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack2(v[2 * e], v[2 * e + 1], inv_l);
-          tmem_st16(t.t_row + C::kTmemS0 + 48 * t.half + 16 * c, pk);
+          tmem_st16(t.t_row + C::kTmemS0 + (kDcT / 4) * t.half + 16 * c, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -720,21 +723,22 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
   }
 }
 
+template <int kDcT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_chunk_attn(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
                  const __grid_constant__ RopeTable tab) {
-  attn_body<kKindMla>(maps, p, &tab);
+  attn_body<kKindMla, kDcT>(maps, p, &tab);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_dense_attn(const __grid_constant__ DenseMaps maps, const __grid_constant__ AttnParams p) {
-  attn_body<kKindDense>(maps, p, nullptr);
+  attn_body<kKindDense, kDc>(maps, p, nullptr);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_mat_attn(const __grid_constant__ MatMaps maps, const __grid_constant__ AttnParams p,
                const __grid_constant__ RopeTable tab) {
-  attn_body<kKindMat>(maps, p, &tab);
+  attn_body<kKindMat, kDc>(maps, p, &tab);
 }
 
 // ---------------------------------------------------------------------------
@@ -792,28 +796,33 @@ bool make_head_map(CUtensorMap* m, const uint16_t* t, int batch, int64_t n_rows,
 
 }  // namespace
 
-cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
-                                   const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
-                                   int heads, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
-                                   int grid_w, float scale, uint16_t* out, int* status,
-                                   cudaStream_t stream, bool* encode_failed) {
+namespace {
+
+template <int kDcT>
+cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                     const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q, int heads,
+                                     int64_t cap, int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale,
+                                     uint16_t* out, int* status, cudaStream_t stream, bool* encode_failed) {
+  using C = Cfg<kKindMla, kDcT>;
+  using L = Layout<kKindMla, kDcT>;
+  constexpr int kRow = kDcT + kDr;
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_chunk_attn, Layout<kKindMla>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  if (!set_smem_attr((const void*)k_chunk_attn<kDcT>, L::kBytes, attr_done)) return cudaErrorInvalidValue;
   ChunkMaps maps;
   bool ok = make_head_map(&maps.q, q, batch, n_q, heads);
   {
-    const cuuint64_t dims[2] = {(cuuint64_t)kDc, (cuuint64_t)heads * kDh};
-    const cuuint64_t strides[1] = {(cuuint64_t)kDc * 2};
+    const cuuint64_t dims[2] = {(cuuint64_t)kDcT, (cuuint64_t)heads * kDh};
+    const cuuint64_t strides[1] = {(cuuint64_t)kDcT * 2};
     const cuuint32_t box[2] = {64, 128};
     ok = ok && make_map(&maps.wuk, w_uk, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&maps.wuv, w_uv, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)kDrow, (cuuint64_t)n_kv, (cuuint64_t)batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)kDrow * 2, (cuuint64_t)cap * kDrow * 2};
-    const cuuint32_t box_c[3] = {64, (cuuint32_t)Cfg<kKindMla>::kBN, 1};
-    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<kKindMla>::kBN, 1};
+    const cuuint64_t dims[3] = {(cuuint64_t)kRow, (cuuint64_t)n_kv, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)kRow * 2, (cuuint64_t)cap * kRow * 2};
+    const cuuint32_t box_c[3] = {64, (cuuint32_t)C::kBN, 1};
+    const cuuint32_t box_r[3] = {32, (cuuint32_t)C::kBN, 1};
     ok = ok && make_map(&maps.c, cache, 3, dims, strides, box_c, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&maps.kr, cache, 3, dims, strides, box_r, CU_TENSOR_MAP_SWIZZLE_64B);
   }
@@ -830,7 +839,7 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + Cfg<kKindMla>::kBN - 1) / Cfg<kKindMla>::kBN);
+  p.n_kv_tiles = (int)((n_kv + C::kBN - 1) / C::kBN);
   p.grid_h = grid_h;
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -838,8 +847,34 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_chunk_attn<<<grid, kThreads, Layout<kKindMla>::kBytes, stream>>>(maps, p, tab);
+  k_chunk_attn<kDcT><<<grid, kThreads, L::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// d_c in {64, 128, 192, 256}; the caller has validated it.
+cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                   const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
+                                   int heads, int d_c, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
+                                   int grid_w, float scale, uint16_t* out, int* status,
+                                   cudaStream_t stream, bool* encode_failed) {
+  switch (d_c) {
+    case 64:
+      return launch_chunk_attention_t<64>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
+                                          grid_w, scale, out, status, stream, encode_failed);
+    case 128:
+      return launch_chunk_attention_t<128>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
+                                           grid_w, scale, out, status, stream, encode_failed);
+    case 192:
+      return launch_chunk_attention_t<192>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
+                                           grid_w, scale, out, status, stream, encode_failed);
+    case 256:
+      return launch_chunk_attention_t<256>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
+                                           grid_w, scale, out, status, stream, encode_failed);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int batch,

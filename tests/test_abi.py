@@ -80,6 +80,18 @@ def test_attention_validation(vm):
     assert L.vmla_selftest_wait_timeout(10, None) == 1
 
 
+def test_latent_width_validation(vm):
+    L = vm.lib
+    f = ctypes.c_float
+    assert L.vmla_cache_append_dc(A, A, A, 1, 10, 1536, 96, A, 100, 0, 0, 8, 8, None) == 2       # d_c
+    assert L.vmla_cache_append_dc(A, A, A, 1, 10, 1536, 320, A, 100, 0, 0, 8, 8, None) == 2      # d_c
+    assert "d_c" in vm.vmla_last_error()
+    assert L.vmla_cache_append_dc(A, A, A, 1, 10, 1500, 64, A, 100, 0, 0, 8, 8, None) == 2       # d_model
+    assert L.vmla_chunk_attention_dc(A, A, A, A, A, 1, 192, 12, 160, 576, 576, 6, 8, 8, f(0.1), A, None) == 2
+    assert "d_c" in vm.vmla_last_error()
+    assert L.vmla_chunk_attention_dc(A, A, A, A, None, 1, 192, 12, 64, 576, 576, 6, 8, 8, f(0.1), A, None) == 1
+
+
 def test_projection_validation(vm):
     L = vm.lib
     assert L.vmla_query_projection(A, A, A, 1, 192, 1536, 12, A, None, None) == 1
