@@ -14,10 +14,11 @@
 // then rounded to bf16 (nearest even).  This is CUDA-core work: the tensor
 // cores do not specify their accumulation order.
 //
-// Tiling: a CTA owns 32 tokens (16 at d_c = 256, to stay within the register
-// budget) x all d_c + 32 outputs; each of its 4 warps owns a quarter of the
-// tokens, and lane l owns outputs l + 32 i, so the rope dims (the last 32
+// Tiling: a CTA owns 32 tokens x all d_c + 32 outputs; each of its 8 warps owns
+// 4 tokens, and lane l owns outputs l + 32 i, so the rope dims (the last 32
 // outputs) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
+// Eight warps (two per scheduler) keep the FMA pipe fed through shared-memory
+// latency; 32 tokens per CTA keep 480P's 4680-token chunk at one CTA per SM.
 // Operands are staged per 64-wide k chunk in shared memory as fp32, double
 // buffered: the global loads of chunk c+1 are issued into registers before the
 // FMAs of chunk c, and land in the other buffer after them, so their latency
@@ -31,14 +32,19 @@ namespace vmla {
 
 namespace {
 constexpr int kKc = 64;          // k chunk
-constexpr int kThreads = 128;    // 4 warps
 constexpr int kStride = kKc + 4; // fp32 row stride in shared memory (conflict-free float4 reads)
 
+// A CTA owns 32 tokens x all d_c + 32 outputs.  Each warp owns 32 / kWarps
+// tokens; lane l owns outputs l + 32 i.  Eight warps (two per scheduler, 4 tokens
+// each) measured fastest for d_c >= 128; at d_c = 64 (three outputs per lane)
+// four warps of 8 tokens reuse each loaded W value over more tokens and win.
 template <int kDcT>
 struct AppendCfg {
   static constexpr int kRow = kDcT + kDr;                    // cached scalars per token
-  static constexpr int kTokPerWarp = kDcT > 192 ? 4 : 8;
-  static constexpr int kTok = 4 * kTokPerWarp;               // tokens per CTA
+  static constexpr int kWarps = kDcT == 64 ? 4 : 8;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kTok = 32;                            // tokens per CTA
+  static constexpr int kTokPerWarp = kTok / kWarps;          // 8 or 4
   static constexpr int kOutPerLane = kRow / 32;              // 3, 5, 7, 9
   static constexpr int kBufFloats = (kRow + kTok) * kStride;
   static constexpr int kSmemBytes = 2 * kBufFloats * 4;
@@ -47,6 +53,38 @@ struct AppendCfg {
   static_assert(kRow % 32 == 0 && (kRow * 8) % kThreads == 0 && (kTok * 8) % kThreads == 0, "tiling");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
+
+// One 4-wide k step of a thread's kO outputs for its kT tokens.  x is stored
+// rotated within each group of four (k+3, k, k+1, k+2), so the two operands of an
+// FMA never sit in the same component of their vectors (fewer register-bank
+// conflicts).  Every accumulator takes k, k+1, k+2, k+3 in turn (its sequential
+// order), and consecutive FMAs belong to different accumulators.
+template <int kT, int kO>
+__device__ __forceinline__ void fma_step(float (&acc)[kT][kO], const float* ws, const float* xs, int lane,
+                                         int tok_row0, int kk) {
+  float4 wv[kO];
+#pragma unroll
+  for (int i = 0; i < kO; ++i) wv[i] = *reinterpret_cast<const float4*>(ws + (lane + 32 * i) * kStride + kk);
+  float4 xv[kT];
+#pragma unroll
+  for (int t = 0; t < kT; ++t) xv[t] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kStride + kk);
+#pragma unroll
+  for (int t = 0; t < kT; ++t)
+#pragma unroll
+    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].y, wv[i].x, acc[t][i]);  // k
+#pragma unroll
+  for (int t = 0; t < kT; ++t)
+#pragma unroll
+    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].z, wv[i].y, acc[t][i]);  // k + 1
+#pragma unroll
+  for (int t = 0; t < kT; ++t)
+#pragma unroll
+    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].w, wv[i].z, acc[t][i]);  // k + 2
+#pragma unroll
+  for (int t = 0; t < kT; ++t)
+#pragma unroll
+    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].x, wv[i].w, acc[t][i]);  // k + 3
+}
 
 struct AppendParams {
   const uint16_t* x;
@@ -67,11 +105,11 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float4& lo, float4
 }
 
 template <int kDcT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(AppendCfg<kDcT>::kThreads, 1)
     k_cache_append(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
   using A = AppendCfg<kDcT>;
   constexpr int kDrow = A::kRow, kTok = A::kTok, kTokPerWarp = A::kTokPerWarp, kOutPerLane = A::kOutPerLane;
-  constexpr int kBufFloats = A::kBufFloats, kWVec = A::kWVec, kXVec = A::kXVec;
+  constexpr int kBufFloats = A::kBufFloats, kWVec = A::kWVec, kXVec = A::kXVec, kThreads = A::kThreads;
   extern __shared__ __align__(16) float smem_f[];
   const int b = blockIdx.y;
   const int tok0 = blockIdx.x * kTok;
@@ -123,8 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = v >> 3, kk = (v & 7) * 8;
       float4 lo, hi;
       bf16x8_to_f32(xreg[n], lo, hi);
-      *reinterpret_cast<float4*>(xs + t * kStride + kk) = lo;
-      *reinterpret_cast<float4*>(xs + t * kStride + kk + 4) = hi;
+      *reinterpret_cast<float4*>(xs + t * kStride + kk) = make_float4(lo.w, lo.x, lo.y, lo.z);
+      *reinterpret_cast<float4*>(xs + t * kStride + kk + 4) = make_float4(hi.w, hi.x, hi.y, hi.z);
     }
   };
 
@@ -136,52 +174,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* ws = smem_f + (c & 1) * kBufFloats;
     const float* xs = ws + kDrow * kStride;
     if (c + 1 < n_chunks) load_chunk((c + 1) * kKc);
-#pragma unroll 1
-    for (int kk = 0; kk < kKc; kk += 4) {
-      float4 wv[kOutPerLane];
-#pragma unroll
-      for (int i = 0; i < kOutPerLane; ++i)
-        wv[i] = *reinterpret_cast<const float4*>(ws + (lane + 32 * i) * kStride + kk);
-#pragma unroll
-      for (int t = 0; t < kTokPerWarp; ++t) {
-        const float4 xv = *reinterpret_cast<const float4*>(xs + (warp * kTokPerWarp + t) * kStride + kk);
-#pragma unroll
-        for (int i = 0; i < kOutPerLane; ++i) {
-          float a = acc[t][i];
-          a = fmaf(xv.x, wv[i].x, a);  // k
-          a = fmaf(xv.y, wv[i].y, a);  // k + 1
-          a = fmaf(xv.z, wv[i].z, a);  // k + 2
-          a = fmaf(xv.w, wv[i].w, a);  // k + 3
-          acc[t][i] = a;
-        }
-      }
-    }
+#pragma unroll 2
+    for (int kk = 0; kk < kKc; kk += 4) fma_step(acc, ws, xs, lane, warp * kTokPerWarp, kk);
     if (c + 1 < n_chunks) store_chunk(smem_f + ((c + 1) & 1) * kBufFloats);
     __syncthreads();
   }
 
-  // 3D rotary embedding of the rope dims (output d_c + lane, the lane's last output).
-  const int pair = lane >> 1;
-  const bool even = (lane & 1) == 0;
-  const int per_frame = p.grid_h * p.grid_w;
+  // 3D rotary embedding of the rope dims: output d_c + lane is the lane's last output.
+  constexpr int kRope = kOutPerLane - 1;
+  {
+    const int pair = lane >> 1;
+    const bool even = (lane & 1) == 0;
+    const int per_frame = p.grid_h * p.grid_w;
 #pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t) {
-    const int tok = tok0 + warp * kTokPerWarp + t;
-    const float v = acc[t][kOutPerLane - 1];
-    const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-    if (tok < p.n_tok) {
-      const int f = tok / per_frame;
-      const int rem = tok - f * per_frame;
-      const int row = rem / p.grid_w;
-      const int col = rem - row * p.grid_w;
-      float2 cs;
-      if (pair < kPairsT) cs = tab.t[f][pair];
-      else if (pair < kPairsT + kPairsH) cs = tab.h[row][pair - kPairsT];
-      else cs = tab.w[col][pair - kPairsT - kPairsH];
-      const float a = even ? v : other;
-      const float bb = even ? other : v;
-      acc[t][kOutPerLane - 1] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
-                                     : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
+    for (int t = 0; t < kTokPerWarp; ++t) {
+      const int tok = tok0 + warp * kTokPerWarp + t;
+      const float v = acc[t][kRope];
+      const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+      if (tok < p.n_tok) {
+        const int f = tok / per_frame;
+        const int rem = tok - f * per_frame;
+        const int row = rem / p.grid_w;
+        const int col = rem - row * p.grid_w;
+        float2 cs;
+        if (pair < kPairsT) cs = tab.t[f][pair];
+        else if (pair < kPairsT + kPairsH) cs = tab.h[row][pair - kPairsT];
+        else cs = tab.w[col][pair - kPairsT - kPairsH];
+        const float a = even ? v : other;
+        const float bb = even ? other : v;
+        acc[t][kRope] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
+                             : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
+      }
     }
   }
 
@@ -222,7 +245,7 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
   const int per_frame = p.grid_h * p.grid_w;
   build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
   dim3 grid((p.n_tok + A::kTok - 1) / A::kTok, batch);
-  k_cache_append<kDcT><<<grid, kThreads, A::kSmemBytes, stream>>>(p, tab);
+  k_cache_append<kDcT><<<grid, A::kThreads, A::kSmemBytes, stream>>>(p, tab);
   return cudaGetLastError();
 }
 }  // namespace
