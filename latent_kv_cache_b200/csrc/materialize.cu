@@ -7,9 +7,16 @@
 // chunk, it lets every denoising step of that chunk run a d = 128 + 32
 // attention over explicit keys instead of the absorbed d = 224 + 192 one.
 //
-// One CTA = 128 keys x one head: D[128 x 256] = C[128 x 192] . [W_UK_h ; W_UV_h]^T
-// (12 tcgen05 MMAs, N = 256, operands staged by TMA), then a bf16 epilogue that
+// Persistent kernel: CTA g takes a contiguous range of work items (sample, head,
+// 128-key tile), ordered head-major so W_UK_h / W_UV_h are loaded once per head
+// and stay in shared memory.  Per item: D[128 keys x 256] = C[128 x 192] .
+// [W_UK_h ; W_UV_h]^T (12 tcgen05 MMAs, N = 256), then a bf16 epilogue that
 // writes K_h to heads [0, H) and V_h to heads [H, 2H) of kv[B, n_kv, 2H, 128].
+// 192 threads: warp 0 TMA producer (the C tiles through a 2-stage ring, W at each
+// head change), warp 1 TMEM allocation + the MMA thread, warps 2-5 the epilogue.
+// TMEM holds two 256-column accumulators, so an item's stores overlap the next
+// item's MMAs.  The epilogue stages each 64-column block of its 32 rows in shared
+// memory and writes it back four full 128-byte lines per store instruction.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -19,14 +26,27 @@
 namespace vmla {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;
+constexpr int kCStages = 2;
 constexpr uint32_t kBlk = 128 * 128;        // 128 rows x 128 B, 128B swizzle
-constexpr uint32_t kA = 0;                  // C tile: 3 blocks (latent 0-63, 64-127, 128-191)
-constexpr uint32_t kB = 3 * kBlk;           // [W_UK_h ; W_UV_h]: per latent block 256 rows
-constexpr uint32_t kBBlk = 2 * kBlk;        // one latent block of B (256 rows)
-constexpr uint32_t kBar = kB + 3 * kBBlk;   // 147456
-constexpr uint32_t kSmemBytes = kBar + 64 + 1024;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kCBytes = 3 * kBlk;      // C tile: 3 blocks (latent 0-63, 64-127, 128-191)
+constexpr uint32_t kBBlk = 2 * kBlk;        // one latent block of [W_UK_h ; W_UV_h] (256 rows)
+constexpr uint32_t kW = 0;                  // W: 3 latent blocks of 256 rows
+constexpr uint32_t kC0 = 3 * kBBlk;         // C ring
+constexpr uint32_t kBar = kC0 + kCStages * kCBytes;  // 196608
+// Epilogue staging: per epilogue warp, 32 rows x 64 bf16 (128 B) padded to 144 B
+// so that row-per-lane writes hit distinct banks.
+constexpr uint32_t kStgRow = 144;
+constexpr uint32_t kStgWarp = 32 * kStgRow;
+constexpr uint32_t kStg = kBar + 256;
+constexpr uint32_t kSmemBytes = kStg + 4 * kStgWarp + 1024;
+constexpr uint32_t kTmemCols = 512;         // two 256-column accumulators
+
+enum {
+  M_CFULL0 = 0, M_CEMPTY0 = kCStages, M_WFULL = 2 * kCStages, M_WEMPTY, M_ACCF0, M_ACCE0 = M_ACCF0 + 2,
+  M_DRAIN = M_ACCE0 + 2, M_COUNT
+};
+static_assert(8 * M_COUNT + 8 <= 256, "barrier area");
 
 struct MatParams {
   uint16_t* kv;  // [B, n_kv, 2H, 128]
@@ -34,6 +54,8 @@ struct MatParams {
   uint64_t wait_limit_ns;
   int64_t n_kv;
   int heads;
+  int n_tiles;   // key tiles per (sample, head)
+  int n_items;   // batch * heads * n_tiles
 };
 
 struct MatGemmMaps {
@@ -42,6 +64,8 @@ struct MatGemmMaps {
   CUtensorMap wuv;
 };
 
+__device__ __forceinline__ uint32_t mbar(uint32_t base, int i) { return base + 8u * i; }
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_materialize_kv(const __grid_constant__ MatGemmMaps maps, const __grid_constant__ MatParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -49,21 +73,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t pad = (uint32_t)(((raw + 1023) & ~uintptr_t(1023)) - raw);
   uint8_t* smem = smem_raw + pad;  // kSmemBytes reserves 1024 B of slack for this
   const uint32_t base = smem_u32(smem);
-  const uint32_t bar_full = base + kBar, bar_mma = base + kBar + 8;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBar + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBar + 20);
+  const uint32_t bars = base + kBar;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBar + 8 * M_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kv0 = blockIdx.x * 128;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // This CTA's items: [it0, it1), item = ((b * heads + h) * n_tiles + tile).
+  const int it0 = (int)((int64_t)p.n_items * blockIdx.x / gridDim.x);
+  const int it1 = (int)((int64_t)p.n_items * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
-    mbar_init(bar_mma, 1);
+    for (int s = 0; s < kCStages; ++s) {
+      mbar_init(mbar(bars, M_CFULL0 + s), 1);
+      mbar_init(mbar(bars, M_CEMPTY0 + s), 1);
+    }
+    mbar_init(mbar(bars, M_WFULL), 1);
+    mbar_init(mbar(bars, M_WEMPTY), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(mbar(bars, M_ACCF0 + a), 1);
+      mbar_init(mbar(bars, M_ACCE0 + a), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(mbar(bars, M_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
@@ -73,50 +106,112 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
 
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_full, 3 * kBlk + 3 * kBBlk);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ producer ------------------------------
+      tma_prefetch_desc(&maps.c);
+      tma_prefetch_desc(&maps.wuk);
+      tma_prefetch_desc(&maps.wuv);
+      int last_c[kCStages] = {-1, -1};
+      int wloads = 0, cur_bh = -1;
+      bool ok = true;
+      for (int it = it0; it < it1 && ok; ++it) {
+        const int bh = it / p.n_tiles, tile = it - bh * p.n_tiles;
+        const int b = bh / p.heads, h = bh - b * p.heads;
+        if (bh != cur_bh) {  // new head: W_UK_h / W_UV_h, once the old ones are no longer read
+          if (wloads > 0 && !(ok = mbar_wait(mbar(bars, M_WEMPTY), (wloads - 1) & 1, ctl, kDevTimeoutProducer)))
+            break;
+          const uint32_t wb = mbar(bars, M_WFULL);
+          mbar_arrive_expect_tx(wb, 3 * kBBlk);
 #pragma unroll
-    for (int blk = 0; blk < 3; ++blk) {
-      tma_load_3d(base + kA + blk * kBlk, &maps.c, bar_full, 64 * blk, kv0, b);
-      tma_load_2d(base + kB + blk * kBBlk, &maps.wuk, bar_full, 64 * blk, h * kDh);
-      tma_load_2d(base + kB + blk * kBBlk + kBlk, &maps.wuv, bar_full, 64 * blk, h * kDh);
+          for (int blk = 0; blk < 3; ++blk) {
+            tma_load_2d(base + kW + blk * kBBlk, &maps.wuk, wb, 64 * blk, h * kDh);
+            tma_load_2d(base + kW + blk * kBBlk + kBlk, &maps.wuv, wb, 64 * blk, h * kDh);
+          }
+          ++wloads;
+          cur_bh = bh;
+        }
+        const int i = it - it0, st = i % kCStages, use = i / kCStages;
+        if (use > 0 && !(ok = mbar_wait(mbar(bars, M_CEMPTY0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer)))
+          break;
+        const uint32_t fb = mbar(bars, M_CFULL0 + st);
+        mbar_arrive_expect_tx(fb, kCBytes);
+#pragma unroll
+        for (int blk = 0; blk < 3; ++blk)
+          tma_load_3d(base + kC0 + st * kCBytes + blk * kBlk, &maps.c, fb, 64 * blk, tile * 128, b);
+        last_c[st] = use;
+      }
+      if (!ok) {  // copies already issued must land before the CTA exits
+        if (wloads > 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(mbar(bars, M_WFULL), (wloads - 1) & 1) && globaltimer_ns() - t0 < p.wait_limit_ns) {
+          }
+        }
+        for (int s = 0; s < kCStages; ++s) {
+          if (last_c[s] < 0) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(mbar(bars, M_CFULL0 + s), last_c[s] & 1) && globaltimer_ns() - t0 < p.wait_limit_ns) {
+          }
+        }
+      }
     }
-    ok = mbar_wait(bar_full, 0, ctl, kDevTimeoutMma);
-    if (ok) {
-      tc_fence_after();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------- MMA --------------------------------
       constexpr uint32_t kId = idesc_bf16_f32(128, 256, false, false);
+      int wsegs = 0, cur_bh = -1;
+      bool ok = true;
+      for (int it = it0; it < it1 && ok; ++it) {
+        const int i = it - it0, st = i % kCStages, acc = i & 1;
+        const int bh = it / p.n_tiles;
+        if (bh != cur_bh) {
+          if (!(ok = mbar_wait(mbar(bars, M_WFULL), wsegs & 1, ctl, kDevTimeoutMma))) break;
+          ++wsegs;
+          cur_bh = bh;
+        }
+        if (i >= 2 && !(ok = mbar_wait(mbar(bars, M_ACCE0 + acc), ((i >> 1) - 1) & 1, ctl, kDevTimeoutMma))) break;
+        if (!(ok = mbar_wait(mbar(bars, M_CFULL0 + st), (i / kCStages) & 1, ctl, kDevTimeoutMma))) break;
+        tc_fence_after();
+        const uint32_t cs = base + kC0 + st * kCBytes;
 #pragma unroll
-      for (int k = 0; k < 12; ++k) {
-        const uint32_t off = (k & 3) * 32;
-        const uint64_t a = smem_desc(base + kA + (k >> 2) * kBlk + off, 16, 1024, kSw128);
-        const uint64_t bd = smem_desc(base + kB + (k >> 2) * kBBlk + off, 16, 1024, kSw128);
-        umma_ss(tmem, a, bd, kId, k > 0);
+        for (int k = 0; k < 12; ++k) {
+          const uint32_t off = (k & 3) * 32;
+          const uint64_t a = smem_desc(cs + (k >> 2) * kBlk + off, 16, 1024, kSw128);
+          const uint64_t bd = smem_desc(base + kW + (k >> 2) * kBBlk + off, 16, 1024, kSw128);
+          umma_ss(tmem + (uint32_t)(acc * 256), a, bd, kId, k > 0);
+        }
+        umma_commit(mbar(bars, M_CEMPTY0 + st));
+        umma_commit(mbar(bars, M_ACCF0 + acc));
+        // Last item of this head: W may be replaced once these MMAs are done.
+        if (it + 1 == it1 || (it + 1) / p.n_tiles != bh) umma_commit(mbar(bars, M_WEMPTY));
       }
-      umma_commit(bar_mma);
-    } else {
-      // The copies issued above must land before the CTA exits.
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bar_full, 0) && globaltimer_ns() - t0 < p.wait_limit_ns) {
+      if (!ok) {
+        umma_commit(mbar(bars, M_DRAIN));
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(mbar(bars, M_DRAIN), 0) && globaltimer_ns() - t0 < p.wait_limit_ns) {
+        }
       }
     }
-  }
-  // Epilogue: thread = key row; TMEM lanes of warp w are rows 32 w .. 32 w + 31.
-  const bool ok_all = mbar_wait(bar_mma, 0, ctl, kDevTimeoutSoftmax);
-  if (__all_sync(0xffffffffu, ok_all)) {
-    tc_fence_after();
-    const int r = warp * 32 + lane;
-    const int64_t j = (int64_t)kv0 + r;
-    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t v[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {  // columns 0-127: K_h, 128-255: V_h
-      tmem_ld32(t_row + 32 * c, v);
-      tmem_ld_wait();
-      if (j < p.n_kv) {
-        const int head = c < 4 ? h : p.heads + h;
-        uint4* dst = reinterpret_cast<uint4*>(
-            p.kv + (((int64_t)b * p.n_kv + j) * (2 * p.heads) + head) * kDh + 32 * (c & 3));
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    // Thread = key row; TMEM lanes of warp w (w % 4 = lane quadrant) are rows 32 (w % 4) ...
+    const int qd = warp & 3;
+    for (int it = it0; it < it1; ++it) {
+      const int i = it - it0, acc = i & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(mbar(bars, M_ACCF0 + acc), (i >> 1) & 1, ctl,
+                                                        kDevTimeoutSoftmax));
+      if (!ok) break;
+      tc_fence_after();
+      const int bh = it / p.n_tiles, tile = it - bh * p.n_tiles;
+      const int b = bh / p.heads, h = bh - b * p.heads;
+      const uint32_t t_row = tmem + (uint32_t)(acc * 256) + ((uint32_t)(qd * 32) << 16);
+      uint8_t* stg = smem + kStg + (warp - 2) * kStgWarp;  // this warp's staging rows
+      const int64_t j0 = (int64_t)tile * 128 + qd * 32;   // first key row of this warp
+      uint32_t v[32];
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {  // 32-column chunks: 0-3 are K_h, 4-7 are V_h
+        tmem_ld32(t_row + 32 * c, v);
+        tmem_ld_wait();
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint4 w;
@@ -124,20 +219,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3]));
           w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5]));
           w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
-          dst[q4] = w;
+          *reinterpret_cast<uint4*>(stg + lane * kStgRow + (c & 1) * 64 + q4 * 16) = w;
+        }
+        if (c & 1) {  // a 64-column block of 32 rows is staged: write it as whole lines
+          __syncwarp();
+          const int head = c < 4 ? h : p.heads + h;
+          const int col0 = ((c >> 1) & 1) * 64;  // 0 or 64 within the head's 128 values
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int idx = lane + 32 * m, row = idx >> 3, q = idx & 7;
+            const int64_t jr = j0 + row;
+            if (jr < p.n_kv) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + row * kStgRow + q * 16);
+              *reinterpret_cast<uint4*>(p.kv + (((int64_t)b * p.n_kv + jr) * (2 * p.heads) + head) * kDh + col0 +
+                                        q * 8) = val;
+            }
+          }
+          __syncwarp();
         }
       }
-    }
-  } else if (threadIdx.x == 0 && ok) {
-    // MMAs were issued but the epilogue gave up: let them finish before TMEM is freed.
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar_mma, 0) && globaltimer_ns() - t0 < p.wait_limit_ns) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mbar(bars, M_ACCE0 + acc));  // accumulator `acc` may be overwritten
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
-    __syncwarp();
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -198,8 +307,14 @@ cudaError_t launch_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, co
     *encode_failed = true;
     return cudaErrorInvalidValue;
   }
-  MatParams p{kv, status, kWaitLimitNs, n_kv, heads};
-  dim3 grid((unsigned)((n_kv + 127) / 128), (unsigned)heads, (unsigned)batch);
+  const int n_tiles = (int)((n_kv + 127) / 128);
+  const int64_t items = (int64_t)batch * heads * n_tiles;
+  if (items > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  static int sms[64] = {0};
+  if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidDevice;
+  MatParams p{kv, status, kWaitLimitNs, n_kv, heads, n_tiles, (int)items};
+  const int grid = items < sms[dev] ? (int)items : sms[dev];  // one CTA per SM (shared memory, TMEM)
   k_materialize_kv<<<grid, kThreads, kSmemBytes, stream>>>(maps, p);
   return cudaGetLastError();
 }
