@@ -495,34 +495,59 @@ def run_ours(args, w, rank, world, local_rank):
     }
     del wq, wqr, wo, q_p, qr_p, y_p
 
-    # ---- end to end through the public API: pinned host inputs -> device -> host result
+    # ---- end to end through the public API: pinned host inputs -> device -> host result.
+    # Every step copies its own inputs in (x of the chunk, q, q_rope) and its output
+    # out.  The step's device tensors are double-buffered so that, as in a serving
+    # loop, step k+1's host-to-device copies and step k-1's device-to-host copy run
+    # on two copy streams while step k computes.
     h_x = x_chunk.cpu().pin_memory()
     h_q = q.cpu().pin_memory()
     h_qr = qr.cpu().pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
     h2d = h_x.numel() * 2 + h_q.numel() * 2 + h_qr.numel() * 2
-    d2h = h_out.numel() * 2
+    d2h = h_out[0].numel() * 2
+    dbuf = [{"x": x_chunk, "q": q, "qr": qr, "out": out},
+            {"x": torch.empty_like(x_chunk), "q": torch.empty_like(q), "qr": torch.empty_like(qr),
+             "out": torch.empty_like(out)}]
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        x_chunk.copy_(h_x, non_blocking=True)
-        q.copy_(h_q, non_blocking=True)
-        qr.copy_(h_qr, non_blocking=True)
-        step()
-        h_out.copy_(out, non_blocking=True)
-
-    for _ in range(args.warmup):
+    def e2e_issue(k):
+        i = k & 1
+        d = dbuf[i]
+        with torch.cuda.stream(s_h2d):
+            if k >= 2:
+                s_h2d.wait_event(ev_done[i])  # step k-2 has finished reading these inputs
+            d["x"].copy_(h_x, non_blocking=True)
+            d["q"].copy_(h_q, non_blocking=True)
+            d["qr"].copy_(h_qr, non_blocking=True)
+            ev_in[i].record(s_h2d)
+        stream.wait_event(ev_in[i])
+        if k >= 2:
+            stream.wait_event(ev_out[i])  # step k-2's output has reached the host
         flush_buf.zero_()
-        e2e_step()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        vm.vmla_cache_append(d["x"], wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w, stream)
+        vm.vmla_chunk_attention(d["q"], d["qr"], wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                d["out"], stream)
+        ev_done[i].record(stream)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev_done[i])
+            h_out[i].copy_(d["out"], non_blocking=True)
+            ev_out[i].record(s_d2h)
+
+    for k in range(args.warmup):
+        e2e_issue(k)
+    e2e_start, e2e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    e2e_start.record(s_h2d)
     for k in range(args.steps):
-        flush_buf.zero_()
-        e2e_ev[k][0].record(stream)
-        e2e_step()
-        e2e_ev[k][1].record(stream)
+        e2e_issue(args.warmup + k)
+    e2e_end.record(s_d2h)
     barrier()
     vm.vmla_get_device_status(stream)
-    e2e_total = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev), dist, dev)
+    e2e_total = max_over_ranks(e2e_start.elapsed_time(e2e_end), dist, dev)
     e2e_value = job_value(world, args.steps, flops_step, e2e_total)
 
     peak, peak_sust, hbm, peak_src = measured_peaks()
@@ -551,7 +576,8 @@ def run_ours(args, w, rank, world, local_rank):
                    "gbs": (x_chunk.numel() * 2 + 224 * w.d_model * 2 + w.batch * w.n_q * 224 * 2)
                    / (app_mean * 1e-3) / 1e9, "hbm_peak_gbs": hbm},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_total / args.steps},
+                "ms_per_step": e2e_total / args.steps,
+                "pipeline": "double-buffered: next step's H2D and previous step's D2H overlap this step's compute"},
         "gpu_launches": gpu_launches,
         "clocks": clocks,
     }
