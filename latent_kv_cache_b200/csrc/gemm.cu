@@ -20,7 +20,8 @@
 //
 // 192 threads per CTA: warp 0 TMA producer (6-stage ring of [A 128x64 | B 128x64]
 // 128B-swizzled k blocks), warp 1 TMEM allocation (+ the MMA issue in the leader),
-// warps 2-5 the epilogue (TMEM lane = output row).  No multicast anywhere: each
+// warps 2-5 the epilogue (TMEM lane = output row; each 64-column block of a warp's
+// 32 rows is staged in shared memory and stored as whole 128-byte lines).  No multicast anywhere: each
 // CTA loads its own operands and the MMA completions are committed to each CTA's
 // barrier separately.  Every wait is bounded (abort flag + device status word).
 #include <cuda.h>
@@ -40,7 +41,12 @@ constexpr uint32_t kABytes = kHalf * kBK * 2;        // 16 KB
 constexpr uint32_t kBBytes = kHalf * kBK * 2;        // 16 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;  // 32 KB
 constexpr uint32_t kBarOff = kStages * kStageBytes;  // 196608
-constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+// Epilogue staging: per epilogue warp, 32 rows x 64 bf16 (128 B) padded to 144 B
+// so that row-per-lane writes hit distinct banks.
+constexpr uint32_t kStgRow = 144;
+constexpr uint32_t kStgWarp = 32 * kStgRow;
+constexpr uint32_t kStg = kBarOff + 256;
+constexpr uint32_t kSmemBytes = kStg + 4 * kStgWarp + 1024;
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 
 enum {
@@ -281,28 +287,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                         kDevTimeoutSoftmax));
       if (!ok) break;
       tc_fence_after();
-      const int row = (t / p.tiles_n) * kTileM + kHalf * (int)rank + qd * 32 + lane;
+      const int row0 = (t / p.tiles_n) * kTileM + kHalf * (int)rank + qd * 32;  // this warp's first row
       const int ncol0 = (t % p.tiles_n) * kTileN;
       const uint32_t t_row = tmem + (uint32_t)(acc * kTileN) + ((uint32_t)(qd * 32) << 16);
+      uint8_t* stg = smem + kStg + (warp - 2) * kStgWarp;
       uint32_t v[32];
 #pragma unroll 1
       for (int c = 0; c < kTileN / 32; ++c) {
         tmem_ld32(t_row + 32 * c, v);
         tmem_ld_wait();
-        const int col = ncol0 + 32 * c;  // 32 columns never straddle N0 (a multiple of 128)
-        if (row < p.m && col < p.n0 + p.n1) {
-          uint16_t* dst = col < p.n0 ? p.c0 + (int64_t)row * p.ldc0 + col
-                                     : p.c1 + (int64_t)row * p.ldc1 + (col - p.n0);
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]), __uint_as_float(v[8 * q4 + 1]));
-            w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3]));
-            w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5]));
-            w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
-            d4[q4] = w;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]), __uint_as_float(v[8 * q4 + 1]));
+          w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3]));
+          w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5]));
+          w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
+          *reinterpret_cast<uint4*>(stg + lane * kStgRow + (c & 1) * 64 + q4 * 16) = w;
+        }
+        if (c & 1) {  // 64 columns of 32 rows staged: store them as whole lines
+          __syncwarp();
+          const int col = ncol0 + 32 * (c - 1);  // a 64-column block never straddles N0 (a multiple of 128)
+          uint16_t* base_ptr = col < p.n0 ? p.c0 + col : p.c1 + (col - p.n0);
+          const int64_t ld = col < p.n0 ? p.ldc0 : p.ldc1;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int idx = lane + 32 * m, r = idx >> 3, q = idx & 7;
+            if (row0 + r < p.m && col + 8 * q < p.n0 + p.n1) {  // N1 is a multiple of 32
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * kStgRow + q * 16);
+              *reinterpret_cast<uint4*>(base_ptr + (int64_t)(row0 + r) * ld + 8 * q) = val;
+            }
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
