@@ -109,3 +109,36 @@ def test_materialized_attention_b8_sampled(vm):
     got = to_f64(out)[:, rows]
     for b in range(w.batch):
         assert_close(got[b], ref[b], f"materialized b8 sample {b}")
+
+
+def test_materialize_kv_many_heads_per_cta(vm):
+    """Batch 40 of a 144-key window (two key tiles, the second ragged) x 12 heads:
+    960 work items over at most one CTA per SM, so each persistent CTA crosses
+    several (sample, head) boundaries and reloads W_UK_h / W_UV_h each time."""
+    import torch
+    w = workload.CONFIGS["tiny"].with_(batch=40, grid_h=4, grid_w=4, seed=123)
+    assert w.n_kv == 144
+    wts, act, cache, ref_cache = _setup(vm, w, cap_extra=5)
+    kv = torch.full((w.batch, w.n_kv, 2 * w.heads, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_materialize_kv(to_dev(wts["w_uk"]), to_dev(wts["w_uv"]), cache, w.n_kv, kv)
+    vm.vmla_get_device_status()
+    ref = oracle.materialized_kv(wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv)
+    got = to_f64(kv)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3)
+
+
+def test_nonabsorbed_1080p_sampled(vm):
+    import torch
+    w = workload.CONFIGS["1080p"]
+    wts, act, cache, ref_cache = _setup(vm, w)
+    kv = torch.empty(w.batch, w.n_kv, 2 * w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_materialize_kv(to_dev(wts["w_uk"]), to_dev(wts["w_uv"]), cache, w.n_kv, kv)
+    out = torch.empty(w.batch, w.n_q, w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_chunk_attention_materialized(to_dev(act["q"]), to_dev(act["q_rope"]), kv, cache, w.n_kv, w.chunk_t0,
+                                         w.grid_h, w.grid_w, SCALE, out)
+    vm.vmla_get_device_status()
+    rows = sample_rows(w.n_q, 24, seed=13)
+    ref = oracle.chunk_attention(act["q"], act["q_rope"], wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv, w.chunk_t0,
+                                 w.grid_h, w.grid_w, SCALE, rows=rows)
+    assert_close(to_f64(out)[:, rows], ref, "nonabsorbed 1080p")
