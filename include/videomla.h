@@ -14,7 +14,8 @@
  *   - bf16 data are passed as pointers to their 16-bit patterns (uint16_t).
  *   - All tensor pointers are DEVICE pointers, contiguous row-major, 16-byte
  *     aligned.  The caller owns every buffer; the library allocates no device
- *     memory per call.
+ *     memory per call (its only device memory is a status word per device and
+ *     the fixed scratch of vmla_chunk_attention_nonabsorbed_noalloc).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on it and never synchronise, except vmla_get_device_status.
  *   - Argument errors return VMLA_ERR_INVALID_ARG / VMLA_ERR_UNSUPPORTED before
@@ -22,7 +23,8 @@
  *     describes the most recent failure of the calling thread.
  *   - Kernels never trap.  Every internal wait has a time limit; a wait that
  *     runs out records a code that vmla_get_device_status reports.
- *   - Compiled sizes: d_c = 192, d_r = 32, per-head dim 128.  The 32 rope dims
+ *   - Compiled sizes: d_c = 192 (also 64, 128, 256 through the *_dc calls),
+ *     d_r = 32, per-head dim 128.  The 32 rope dims
  *     split into (t: 12, h: 10, w: 10); pair i of an axis with d_a dims turns at
  *     1e4^(-2i/d_a) radians per position; pairs are adjacent dims.
  *   - Token n of a call that starts at frame t0 on a grid_h x grid_w patch grid

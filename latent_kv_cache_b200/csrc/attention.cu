@@ -3,11 +3,11 @@
 //
 // VideoMLA ("Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video
 // Diffusion", abstract; summary "Approach"): keys and values of every head are
-// generated from one head-shared content latent c (192) plus one head-shared
-// rope key k_r (32).  With W_UK absorbed into the query,
+// generated from one head-shared content latent c (d_c = 192 in the paper's
+// model) plus one head-shared rope key k_r (32).  With W_UK absorbed into the query,
 //     score(i, j) = scale * ( (q_h,i W_UK_h) . c_j + RoPE(q_r,h,i) . k_r,j ),
 //     out_h,i     = ( sum_j softmax_j(score) c_j ) W_UV_h^T,
-// so one CTA streams 224-wide cache rows [c ; k_r] and never materialises K or V.
+// so one CTA streams (d_c + 32)-wide cache rows [c ; k_r] and never materialises K or V.
 //
 // One CTA = one 128-query tile of one head of one sample; heads are the fastest
 // grid index so the 12 CTAs that read the same cache tiles run together and
@@ -138,10 +138,10 @@ static_assert(B_COUNT * 8 + 8 <= 512, "barrier area");
 
 struct ChunkMaps {
   CUtensorMap q;    // [B, Nq, H, 128] box (64, 1, 128, 1), 128B swizzle
-  CUtensorMap wuk;  // [H*128, 192]    box (64, 128), 128B swizzle
-  CUtensorMap wuv;  // [H*128, 192]    box (64, 128), 128B swizzle
-  CUtensorMap c;    // [B, n_kv, 224]  box (64, 96, 1), 128B swizzle (content latent)
-  CUtensorMap kr;   // [B, n_kv, 224]  box (32, 96, 1), 64B swizzle (rope key, x = 192)
+  CUtensorMap wuk;  // [H*128, d_c]         box (64, 128), 128B swizzle
+  CUtensorMap wuv;  // [H*128, d_c]         box (64, 128), 128B swizzle
+  CUtensorMap c;    // [B, n_kv, d_c + 32]  box (64, 128, 1), 128B swizzle (content latent)
+  CUtensorMap kr;   // [B, n_kv, d_c + 32]  box (32, 128, 1), 64B swizzle (rope key, x = d_c)
 };
 
 struct DenseMaps {
