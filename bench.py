@@ -595,12 +595,17 @@ def run_ours(args, w, rank, world, local_rank):
 # The full per-chunk schedule: L layers x (1 append + S denoising-step attentions),
 # captured once as a CUDA graph and replayed (timing-only inputs drawn on device)
 # ---------------------------------------------------------------------------
-def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, full_layer=False):
-    """Per-layer latent caches (filled by appends over the cached frames), the
-    chunk's tokens, per-(layer, step) queries and outputs.  Returns a list of
-    zero-argument launch closures in schedule order and the tensors they use.
+def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, full_layer=False, chunks=1):
+    """Per-layer caches (filled by appends over the cached frames), the chunk's
+    tokens, per-(layer, step) queries and outputs.  Returns, for each of `chunks`
+    consecutive chunks, a list of zero-argument launch closures in schedule order,
+    and the tensors they use.  Chunk g starts at frame cached_frames + g * chunk_frames
+    and its tokens go to ring slots (n_cached + g * n_q) mod n_kv: from the second
+    chunk on, each append evicts the window's oldest frames.
     full_layer: each (step, layer) also computes its queries from the hidden
-    states (q, q_r = x W_Q^T, x W_QR^T) and projects the heads' output (o W_O^T)."""
+    states (q, q_r = x W_Q^T, x W_QR^T) and projects the heads' output (o W_O^T).
+    dense: the per-head baseline, whose per-layer append writes the chunk's
+    K = x W_K^T and V = x W_V^T (3072 scalars per token) into its ring."""
     import torch
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
@@ -624,8 +629,12 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, ful
             vm.vmla_cache_append(x_win[:, f0 * per:(f0 + nf) * per].contiguous(), L["wd"], L["wk"], L["cache"],
                                  f0 * per, f0, w.grid_h, w.grid_w)
         if dense:
+            if w.batch != 1 or D != H * w.d_head:
+                raise ValueError("the dense schedule writes K/V slices in place: batch 1, d_model = heads * 128")
             L["k"] = rnd(w.batch, w.n_kv, H, w.d_head)
             L["v"] = rnd(w.batch, w.n_kv, H, w.d_head)
+            L["w_kd"] = rnd(H * w.d_head, D, std=D ** -0.5)
+            L["w_vd"] = rnd(H * w.d_head, D, std=D ** -0.5)
         if full_layer:
             L["wq"] = rnd(H * w.d_head, D, std=D ** -0.5)
             L["wqr"] = rnd(H * w.d_r, D, std=D ** -0.5)
@@ -635,30 +644,42 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, ful
             L["kv"] = torch.empty(w.batch, w.n_kv, 2 * H, w.d_head, dtype=torch.bfloat16, device=dev)
         layers.append(L)
     del x_win
-    ops = []
-    for s in range(w.steps):
-        for L in layers:
-            if dense:
-                ops.append(lambda L=L, s=s: vm.vmla_dense_attention(L["q"][s], L["k"], L["v"], SCALE, L["out"][s]))
-                continue
-            if s == 0:  # the chunk's latents enter the window's tail slots once per layer
-                ops.append(lambda L=L: vm.vmla_cache_append(x_chunk, L["wd"], L["wk"], L["cache"], w.n_cached,
-                                                            w.chunk_t0, w.grid_h, w.grid_w))
+    x_heads = x_chunk.view(w.batch, w.n_q, H, w.d_head) if dense else None
+
+    def chunk_ops(ci):
+        slot = (w.n_cached + ci * w.n_q) % w.n_kv
+        t0 = w.chunk_t0 + ci * w.chunk_frames
+        ops = []
+        for s in range(w.steps):
+            for L in layers:
+                if dense:
+                    if s == 0:  # the chunk's K and V enter the dense ring once per layer
+                        for wn, cn in (("w_kd", "k"), ("w_vd", "v")):
+                            dst = L[cn][:, slot:slot + w.n_q].view(w.batch, w.n_q, D)
+                            ops.append(lambda L=L, wn=wn, dst=dst: vm.vmla_output_projection(x_heads, L[wn], dst))
+                    ops.append(lambda L=L, s=s: vm.vmla_dense_attention(L["q"][s], L["k"], L["v"], SCALE, L["out"][s]))
+                    continue
+                if s == 0:  # the chunk's latents enter the window's ring once per layer
+                    ops.append(lambda L=L: vm.vmla_cache_append(x_chunk, L["wd"], L["wk"], L["cache"], slot, t0,
+                                                                w.grid_h, w.grid_w))
+                    if nonabsorbed:
+                        ops.append(lambda L=L: vm.vmla_materialize_kv(L["wuk"], L["wuv"], L["cache"], w.n_kv, L["kv"]))
                 if nonabsorbed:
-                    ops.append(lambda L=L: vm.vmla_materialize_kv(L["wuk"], L["wuv"], L["cache"], w.n_kv, L["kv"]))
-            if nonabsorbed:
-                ops.append(lambda L=L, s=s: vm.vmla_chunk_attention_materialized(
-                    L["q"][s], L["qr"][s], L["kv"], L["cache"], w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
-                    L["out"][s]))
-                continue
-            if full_layer:
-                ops.append(lambda L=L, s=s: vm.vmla_query_projection(x_chunk, L["wq"], L["wqr"], L["q"][s], L["qr"][s]))
-            ops.append(lambda L=L, s=s: vm.vmla_chunk_attention(L["q"][s], L["qr"][s], L["wuk"], L["wuv"], L["cache"],
-                                                                w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
-                                                                L["out"][s]))
-            if full_layer:
-                ops.append(lambda L=L, s=s: vm.vmla_output_projection(L["out"][s], L["wo"], L["y"]))
-    return ops, layers
+                    ops.append(lambda L=L, s=s: vm.vmla_chunk_attention_materialized(
+                        L["q"][s], L["qr"][s], L["kv"], L["cache"], w.n_kv, t0, w.grid_h, w.grid_w, SCALE,
+                        L["out"][s]))
+                    continue
+                if full_layer:
+                    ops.append(lambda L=L, s=s: vm.vmla_query_projection(x_chunk, L["wq"], L["wqr"], L["q"][s],
+                                                                         L["qr"][s]))
+                ops.append(lambda L=L, s=s: vm.vmla_chunk_attention(L["q"][s], L["qr"][s], L["wuk"], L["wuv"],
+                                                                    L["cache"], w.n_kv, t0, w.grid_h, w.grid_w,
+                                                                    SCALE, L["out"][s]))
+                if full_layer:
+                    ops.append(lambda L=L, s=s: vm.vmla_output_projection(L["out"][s], L["wo"], L["y"]))
+        return ops
+
+    return [chunk_ops(ci) for ci in range(chunks)], layers
 
 
 def capture_graph(ops):
@@ -691,48 +712,44 @@ def run_chunk_schedule(args, w, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    def timed(graph, n):
-        for _ in range(args.warmup):
-            graph.replay()
+    # One graph per ring position: chunk c replays graph c mod G, so consecutive
+    # chunks slide the window (each append evicts the oldest frames).
+    G = w.n_kv // w.n_q if w.n_kv % w.n_q == 0 else 1
+
+    def timed(graphs, n):
+        for i in range(max(args.warmup, len(graphs))):
+            graphs[i % len(graphs)].replay()
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record()
-        for _ in range(n):
-            graph.replay()
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
         ev[1].record()
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         return max_over_ranks(ev[0].elapsed_time(ev[1]) / n, dist, dev)
 
-    ops, _ = build_chunk_schedule(vm, w, dev, seed=1000 + rank)
-    graph = capture_graph(ops)
-    vm.vmla_get_device_status()
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    ms_chunk = timed(graph, args.steps)
-    clocks = sampler.stop()
-    vm.vmla_get_device_status()
-    del graph, ops
-    torch.cuda.empty_cache()
-    ops_n, _ = build_chunk_schedule(vm, w, dev, seed=1000 + rank, nonabsorbed=True)
-    graph_n = capture_graph(ops_n)
-    ms_nonabs = timed(graph_n, args.steps)
-    vm.vmla_get_device_status()
-    del graph_n, ops_n
-    torch.cuda.empty_cache()
-    ops_f, _ = build_chunk_schedule(vm, w, dev, seed=1000 + rank, full_layer=True)
-    graph_f = capture_graph(ops_f)
-    ms_full = timed(graph_f, args.steps)
-    vm.vmla_get_device_status()
-    del graph_f, ops_f
-    torch.cuda.empty_cache()
-    ops_d, _ = build_chunk_schedule(vm, w, dev, seed=2000 + rank, dense=True)
-    graph_d = capture_graph(ops_d)
-    ms_dense = timed(graph_d, args.steps)
-    vm.vmla_get_device_status()
+    def measure(sampler=None, **kind):
+        op_lists, _ = build_chunk_schedule(vm, w, dev, seed=(2000 if kind.get("dense") else 1000) + rank,
+                                           chunks=G, **kind)
+        graphs = [capture_graph(ops) for ops in op_lists]
+        vm.vmla_get_device_status()
+        if sampler is not None:
+            sampler.start()
+        ms = timed(graphs, args.steps)
+        clocks = sampler.stop() if sampler is not None else None
+        vm.vmla_get_device_status()
+        del graphs, op_lists
+        torch.cuda.empty_cache()
+        return ms, clocks
+
+    ms_chunk, clocks = measure(ClockSampler(local_rank))
+    ms_nonabs, _ = measure(nonabsorbed=True)
+    ms_full, _ = measure(full_layer=True)
+    ms_dense, _ = measure(dense=True)
     flops = w.layers * w.steps * w.attention_flops() + w.layers * w.append_flops()
     value = job_value(world, 1, flops, ms_chunk)
     n_launch = w.layers * w.steps + w.layers  # the absorbed graph, whose time is `value`
@@ -742,6 +759,8 @@ def run_chunk_schedule(args, w, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_desc(w), step=f"one chunk: {w.layers} layers x ({w.steps} chunk attentions) "
                                                f"+ {w.layers} cache appends, one CUDA graph replay",
+                       window=f"sliding: {G} graphs (one per ring position) replayed in rotation, each "
+                              f"chunk's append evicts the oldest {w.chunk_frames} frames",
                        l2="inputs larger than L2 (per-layer caches, queries and outputs)"),
         "nonabsorbed": {"ms_per_chunk": ms_nonabs,
                         "transient_kv_bytes": w.layers * w.batch * w.n_kv * 2 * w.heads * w.d_head * 2},
@@ -750,6 +769,7 @@ def run_chunk_schedule(args, w, rank, world, local_rank):
                                "one append per layer",
                        "projection_flops_per_chunk": w.layers * w.steps * w.io_projection_flops()},
         "dense": {"ms_per_chunk": ms_dense, "layers": w.layers, "steps": w.steps,
+                  "append": "K = x W_K^T and V = x W_V^T of the chunk written into the dense ring per layer",
                   "kv_cache_bytes": {"mla": w.layers * w.batch * w.n_kv * 448,
                                      "dense": w.layers * w.batch * w.n_kv * 6144}},
         "gpu_launches": args.steps * n_launch, "clocks": clocks,
