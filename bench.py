@@ -230,15 +230,33 @@ def size_oracle_sample(w, act, wts, cache_bits, target_s):
     return np.linspace(0, w.n_q - 1, n_rows).astype(np.int64), n_tok
 
 
+def dense_oracle_sample(w, kv, act, n_rows):
+    """The fp64 dense per-head oracle on n_rows query rows: seconds and TFLOP/s (2 x 2 x d per score)."""
+    import oracle
+    rows = np.linspace(0, w.n_q - 1, n_rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.dense_attention(act["q"], kv["k"], kv["v"], SCALE, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, w.dense_flops() * len(rows) / w.n_q / dt / 1e12
+
+
 def cpu_baseline(w, act, wts, target_s):
     cache_bits = oracle_prepare(w, act, wts)
     rows, n_tok = size_oracle_sample(w, act, wts, cache_bits, target_s)
     dt, flops = oracle_sample_step(w, act, wts, cache_bits, rows, n_tok)
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+    line = {"value": flops / dt / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
             "sample": (f"fp64 oracle: append of {n_tok} chunk tokens + attention of {len(rows)} of "
                        f"{w.n_q} query rows x {w.heads} heads x {w.n_kv} keys; {dt:.1f} s; FLOPs "
                        f"counted with the same absorbed convention as the GPU value"),
             "seconds": dt}
+    # The dense per-head baseline's oracle, timed the same way on a few seconds' worth of rows.
+    kv = workload.batch_dense_kv(w)
+    d64, _ = dense_oracle_sample(w, kv, act, 64)
+    n_dense = int(min(w.n_q, max(64, 64 * max(1.0, (target_s / 3) / max(d64, 1e-3)))))
+    dd, dense_tf = dense_oracle_sample(w, kv, act, n_dense)
+    line["dense"] = {"value": dense_tf, "unit": "TFLOP/s", "seconds": dd,
+                     "sample": f"fp64 dense oracle: {n_dense} of {w.n_q} query rows x {w.heads} heads x {w.n_kv} keys"}
+    return line
 
 
 # ---------------------------------------------------------------------------
@@ -572,6 +590,7 @@ def run_ours(args, w, rank, world, local_rank):
                      "frac": achieved / peak, "traffic": profiled_traffic(),
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "kernel": "k_chunk_attn"},
+        "attention_dram_read_gbs": (profiled_traffic() / (attn_mean * 1e-3) / 1e9) if profiled_traffic() else None,
         "append": {"us": app_mean * 1e3, "bound": "alu",
                    "gbs": (x_chunk.numel() * 2 + 224 * w.d_model * 2 + w.batch * w.n_q * 224 * 2)
                    / (app_mean * 1e-3) / 1e9, "hbm_peak_gbs": hbm},
