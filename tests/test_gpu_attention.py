@@ -131,14 +131,14 @@ def test_chunk_attention_identical_keys(vm):
 
 def test_chunk_attention_480p_sampled(vm):
     w = workload.CONFIGS["480p"]
-    rows = sample_rows(w.n_q, 192, seed=1)
+    rows = sample_rows(w.n_q, 512, seed=1)
     got, ref = _mla_case(vm, w, rows=rows)
     assert_close(got, ref, "480p")
 
 
 def test_chunk_attention_480p_b8_sampled(vm):
     w = workload.CONFIGS["480p_b8"]
-    rows = sample_rows(w.n_q, 48, seed=2)
+    rows = sample_rows(w.n_q, 64, seed=2)
     got, ref = _mla_case(vm, w, rows=rows)
     assert_close(got, ref, "480p b8")
     # no cross-sample leakage: each sample's rows match its own oracle rows
@@ -148,7 +148,7 @@ def test_chunk_attention_480p_b8_sampled(vm):
 
 def test_chunk_attention_1080p_sampled(vm):
     w = workload.CONFIGS["1080p"]
-    rows = sample_rows(w.n_q, 96, seed=3)
+    rows = sample_rows(w.n_q, 512, seed=3)
     got, ref = _mla_case(vm, w, rows=rows)
     assert_close(got, ref, "1080p")
 
