@@ -458,3 +458,23 @@ def test_planted_dropped_rope_term_is_caught():
     good = oracle.chunk_attention(q, qr, wuk, wuv, cache, 9, 0, 2, 3, 0.5)
     no_rope = oracle.chunk_attention(q, np.zeros_like(qr), wuk, wuv, cache, 9, 0, 2, 3, 0.5)
     assert np.abs(good - no_rope).max() > 1e-4
+
+
+def test_input_generator_bf16_rounding_and_streams():
+    # The seeded input generator (shared by the oracle and the GPU path) rounds to
+    # bf16 like torch's cast, decodes exactly, and gives each named tensor its own
+    # reproducible stream.
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal(50000).astype(np.float32) * np.float32(11.0)
+    ties = (np.arange(1, 1000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    v = np.concatenate([v, ties, -ties])
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(workload.bf16_bits(v), ref)
+    assert np.array_equal(workload.bf16_to_f32(ref), torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16)
+                          .float().numpy())
+    a = workload.normal_bf16(5, (0, 1), (64, 8))
+    assert np.array_equal(a, workload.normal_bf16(5, (0, 1), (64, 8)))
+    assert not np.array_equal(a, workload.normal_bf16(5, (0, 2), (64, 8)))
+    assert not np.array_equal(a, workload.normal_bf16(6, (0, 1), (64, 8)))
+    f = workload.bf16_to_f32(workload.normal_bf16(3, (9,), (200000,), std=0.25)).astype(np.float64)
+    assert abs(f.mean()) < 0.01 and abs(f.std() - 0.25) < 0.005
