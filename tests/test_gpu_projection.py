@@ -141,3 +141,25 @@ def test_layer_chain_480p_sampled(vm):
                                 w.grid_w, SCALE, rows=rows)
     ry = oracle.linear(oracle.round_bf16(ro).reshape(w.batch, len(rows), -1), iw["w_o"])
     assert_close(to_f64(y)[:, rows], ry, "480p layer chain")
+
+
+def test_projections_minimum_shapes(vm):
+    """One token, one head, a single 64-wide k block (query side) and d_model 128
+    (output side): one M tile, one N tile, a one-block pipeline."""
+    import torch
+    rng = np.random.default_rng(41)
+
+    def bits(*shape, std=1.0):
+        return workload.bf16_bits((rng.standard_normal(shape) * std).astype(np.float32))
+
+    x, wq, wqr = bits(1, 1, 64), bits(128, 64, std=0.125), bits(32, 64, std=0.125)
+    q = torch.full((1, 1, 1, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qr = torch.full((1, 1, 1, 32), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_query_projection(to_dev(x), to_dev(wq), to_dev(wqr), q, qr)
+    o, wo = bits(1, 1, 1, 128), bits(128, 128, std=128 ** -0.5)
+    y = torch.full((1, 1, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_output_projection(to_dev(o), to_dev(wo), y)
+    vm.vmla_get_device_status()
+    _check(to_f64(q), oracle.linear(x, wq).reshape(1, 1, 1, 128), "q, one token")
+    _check(to_f64(qr), oracle.linear(x, wqr).reshape(1, 1, 1, 32), "q_rope, one token")
+    _check(to_f64(y), oracle.linear(o.reshape(1, 1, 128), wo), "y, one token")
