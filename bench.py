@@ -90,9 +90,10 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(workload_name: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu summary,
-    or None if the summary is missing or the kernel source changed since."""
+    or None if the summary is missing, covers another workload, or the kernel
+    source changed since."""
     try:
         vals = {}
         with open(PROFILE_SUMMARY) as f:
@@ -100,7 +101,7 @@ def profiled_traffic():
                 if line.startswith("- ") and ":" in line:
                     k, v = line[2:].split(":", 1)
                     vals[k.strip()] = v.strip().strip("`")
-        if vals.get("source_sha256_16") != attn_source_hash():
+        if vals.get("source_sha256_16") != attn_source_hash() or vals.get("workload") != workload_name:
             return None
         return int(vals["dram_bytes_per_launch"])
     except Exception:
@@ -570,6 +571,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     peak, peak_sust, hbm, peak_src = measured_peaks()
     achieved = w.attention_flops() / (attn_mean * 1e-3) / 1e12
+    traffic = profiled_traffic(w.name)
+    sm_max = clocks.get("sm_max_mhz") or 1965
+    fp32_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -587,11 +591,14 @@ def run_ours(args, w, rank, world, local_rank):
                   "mla_over_dense_ms": attn_mean / dense_ms,
                   "cache_bytes_per_token": {"mla": 224 * 2, "dense": 3072 * 2}},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "kernel": "k_chunk_attn"},
-        "attention_dram_read_gbs": (profiled_traffic() / (attn_mean * 1e-3) / 1e9) if profiled_traffic() else None,
+        "attention_dram_read_gbs": (traffic / (attn_mean * 1e-3) / 1e9) if traffic else None,
         "append": {"us": app_mean * 1e3, "bound": "alu",
+                   "fp32_tflops": w.append_flops() / (app_mean * 1e-3) / 1e12,
+                   "fp32_peak_tflops": fp32_peak, "frac": w.append_flops() / (app_mean * 1e-3) / 1e12 / fp32_peak,
+                   "fp32_peak_source": "148 SMs x 128 FMA lanes x 2 flop x the max SM clock",
                    "gbs": (x_chunk.numel() * 2 + 224 * w.d_model * 2 + w.batch * w.n_q * 224 * 2)
                    / (app_mean * 1e-3) / 1e9, "hbm_peak_gbs": hbm},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -2,8 +2,8 @@
 //
 // VideoMLA ("Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video
 // Diffusion", abstract and summary "Approach"): each cached token stores a
-// head-shared content latent (d_c = 192 in the paper's model; the kernel is a
-// template over d_c in {64, 128, 192, 256}) and a head-shared decoupled 3D-RoPE
+// head-shared content latent (d_c = 192 in the paper's model; the kernels are
+// templates over d_c in {64, 128, 192, 256}) and a head-shared decoupled 3D-RoPE
 // key (32).
 //
 // The arithmetic order is fixed so the result is reproducible bit for bit:
@@ -14,15 +14,31 @@
 // then rounded to bf16 (nearest even).  This is CUDA-core work: the tensor
 // cores do not specify their accumulation order.
 //
-// Tiling: a CTA owns 32 tokens x all d_c + 32 outputs; each of its 8 warps owns
-// 4 tokens, and lane l owns outputs l + 32 i, so the rope dims (the last 32
-// outputs) sit one per lane and a pair (2p, 2p+1) lives in lanes (2p, 2p+1).
-// Eight warps (two per scheduler) keep the FMA pipe fed through shared-memory
-// latency; 32 tokens per CTA keep 480P's 4680-token chunk at one CTA per SM.
-// Operands are staged per 64-wide k chunk in shared memory as fp32, double
-// buffered: the global loads of chunk c+1 are issued into registers before the
-// FMAs of chunk c, and land in the other buffer after them, so their latency
-// hides behind the arithmetic.
+// What bounds it.  A CTA owns 32 tokens x all d_c + 32 outputs, and 480P's
+// 4680-token chunk is one such tile per SM.  Shared memory delivers 32 four-byte
+// words per clock whatever the access width or broadcast, so the operand words a
+// thread reads per FMA decide the speed once the FMAs are spread over enough
+// threads to keep the schedulers busy.  Hence:
+//  - W stays bf16 in shared memory (half the words of fp32) and is widened in
+//    registers (exact: a bf16 is the top half of an fp32), one instruction per
+//    W value;
+//  - the FMAs of two outputs of a token are issued as one fma.rn.f32x2 (two
+//    separately rounded fp32 FMAs, the same bits as two fmaf), which frees the
+//    issue slots the widening costs;
+//  - x is widened to fp32 once per CTA when it is staged.
+// Two thread layouts share this scheme:
+//  - wide (8 warps, two per scheduler): warp w owns tokens 4w .. 4w+3, lane l
+//    owns outputs l + 32 i.  Used when each SM holds one tile.
+//  - tall (4 warps): lanes form 4 token groups x 8 output groups and a thread
+//    holds 8 tokens x (d_c + 32) / 32 outputs, half the operand words per FMA of
+//    the wide form.  With one warp per scheduler it stalls more, so it only wins
+//    where two tiles share an SM (more tiles than SMs, d_c <= 192).
+//
+// Operands per 64-wide k chunk: W (d_c + 32 rows of bf16) is copied by
+// cp.async into a 3-stage ring; x (32 rows) is loaded one chunk ahead into
+// registers, widened and stored into a double buffer.  The k steps of a chunk
+// are software pipelined: the loads of step s + 1 are spread over the FMAs of
+// step s.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -31,60 +47,11 @@
 namespace vmla {
 
 namespace {
-constexpr int kKc = 64;          // k chunk
-constexpr int kStride = kKc + 4; // fp32 row stride in shared memory (conflict-free float4 reads)
-
-// A CTA owns 32 tokens x all d_c + 32 outputs.  Each warp owns 32 / kWarps
-// tokens; lane l owns outputs l + 32 i.  Eight warps (two per scheduler, 4 tokens
-// each) measured fastest for d_c >= 128; at d_c = 64 (three outputs per lane)
-// four warps of 8 tokens reuse each loaded W value over more tokens and win.
-template <int kDcT>
-struct AppendCfg {
-  static constexpr int kRow = kDcT + kDr;                    // cached scalars per token
-  static constexpr int kWarps = kDcT == 64 ? 4 : 8;
-  static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kTok = 32;                            // tokens per CTA
-  static constexpr int kTokPerWarp = kTok / kWarps;          // 8 or 4
-  static constexpr int kOutPerLane = kRow / 32;              // 3, 5, 7, 9
-  static constexpr int kBufFloats = (kRow + kTok) * kStride;
-  static constexpr int kSmemBytes = 2 * kBufFloats * 4;
-  static constexpr int kWVec = kRow * 8 / kThreads;          // 16-byte W vectors per thread per chunk
-  static constexpr int kXVec = kTok * 8 / kThreads;          // 16-byte x vectors per thread per chunk
-  static_assert(kRow % 32 == 0 && (kRow * 8) % kThreads == 0 && (kTok * 8) % kThreads == 0, "tiling");
-  static_assert(kSmemBytes <= 232448, "shared memory");
-};
-
-// One 4-wide k step of a thread's kO outputs for its kT tokens.  x is stored
-// rotated within each group of four (k+3, k, k+1, k+2), so the two operands of an
-// FMA never sit in the same component of their vectors (fewer register-bank
-// conflicts).  Every accumulator takes k, k+1, k+2, k+3 in turn (its sequential
-// order), and consecutive FMAs belong to different accumulators.
-template <int kT, int kO>
-__device__ __forceinline__ void fma_step(float (&acc)[kT][kO], const float* ws, const float* xs, int lane,
-                                         int tok_row0, int kk) {
-  float4 wv[kO];
-#pragma unroll
-  for (int i = 0; i < kO; ++i) wv[i] = *reinterpret_cast<const float4*>(ws + (lane + 32 * i) * kStride + kk);
-  float4 xv[kT];
-#pragma unroll
-  for (int t = 0; t < kT; ++t) xv[t] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kStride + kk);
-#pragma unroll
-  for (int t = 0; t < kT; ++t)
-#pragma unroll
-    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].y, wv[i].x, acc[t][i]);  // k
-#pragma unroll
-  for (int t = 0; t < kT; ++t)
-#pragma unroll
-    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].z, wv[i].y, acc[t][i]);  // k + 1
-#pragma unroll
-  for (int t = 0; t < kT; ++t)
-#pragma unroll
-    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].w, wv[i].z, acc[t][i]);  // k + 2
-#pragma unroll
-  for (int t = 0; t < kT; ++t)
-#pragma unroll
-    for (int i = 0; i < kO; ++i) acc[t][i] = fmaf(xv[t].x, wv[i].w, acc[t][i]);  // k + 3
-}
+constexpr int kKc = 64;             // k chunk
+constexpr int kTok = 32;            // tokens per CTA
+constexpr int kXStride = kKc + 8;   // fp32 x row stride in shared memory (72 words)
+constexpr int kWStride = kKc + 8;   // bf16 W row stride in shared memory (144 bytes)
+constexpr int kWStages = 3;
 
 struct AppendParams {
   const uint16_t* x;
@@ -99,153 +66,442 @@ struct AppendParams {
   int grid_w;
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float4& lo, float4& hi) {
-  lo = make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
-  hi = make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
+// Shared-memory plan and staging shares of a layout with kThreads threads.
+template <int kDcT, int kThreads>
+struct Stage {
+  static constexpr int kRow = kDcT + kDr;                    // cached scalars per token
+  static constexpr int kWStageBytes = kRow * kWStride * 2;
+  static constexpr int kXBufFloats = kTok * kXStride;
+  static constexpr int kSmemBytes = kWStages * kWStageBytes + 2 * kXBufFloats * 4;
+  static constexpr int kWCopies = kRow * (kKc / 8) / kThreads;  // 16-byte W copies per thread per chunk
+  static constexpr int kXVec = kTok * (kKc / 8) / kThreads;     // 16-byte x loads per thread per chunk
+  static_assert(kRow % 32 == 0, "rows");
+  static_assert((kRow * (kKc / 8)) % kThreads == 0 && (kTok * (kKc / 8)) % kThreads == 0, "staging");
+  static_assert(kTok * kRow * 2 <= kSmemBytes, "output staging");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kN>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kN) : "memory"); }
+
+__device__ __forceinline__ uint32_t u4comp(const uint4& v, int e) {
+  return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ float f4comp(const float4& v, int e) {
+  return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+}
+// k value e of a bf16 pair word (e even: the low half).
+__device__ __forceinline__ float widen(uint32_t word, int e) {
+  return (e & 1) ? bf16hi_to_f32(word) : bf16lo_to_f32(word);
 }
 
-template <int kDcT>
-__global__ void __launch_bounds__(AppendCfg<kDcT>::kThreads, 1)
-    k_cache_append(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
-  using A = AppendCfg<kDcT>;
-  constexpr int kDrow = A::kRow, kTok = A::kTok, kTokPerWarp = A::kTokPerWarp, kOutPerLane = A::kOutPerLane;
-  constexpr int kBufFloats = A::kBufFloats, kWVec = A::kWVec, kXVec = A::kXVec, kThreads = A::kThreads;
-  extern __shared__ __align__(16) float smem_f[];
-  const int b = blockIdx.y;
-  const int tok0 = blockIdx.x * kTok;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+// The chunk pipeline shared by both layouts: W ring by cp.async, x staged
+// through registers, one __syncthreads per chunk.  `compute(xs, ws)` runs the
+// FMAs of one chunk.
+template <int kDcT, int kThreads, class Compute>
+__device__ __forceinline__ void run_chunks(const AppendParams& p, uint8_t* smem_raw, int b, int tok0,
+                                           Compute&& compute) {
+  using S = Stage<kDcT, kThreads>;
+  uint16_t* wring = reinterpret_cast<uint16_t*>(smem_raw);
+  float* xbuf = reinterpret_cast<float*>(smem_raw + kWStages * S::kWStageBytes);
+  const uint32_t wring_s = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
   const uint16_t* xb = p.x + (int64_t)b * p.n_tok * p.d_model;
+  const int n_chunks = p.d_model / kKc;
 
-  float acc[kTokPerWarp][kOutPerLane];
+  // W chunk c -> ring stage c % kWStages: copy v = threadIdx.x + kThreads * n is
+  // row v / 8, bytes 16 (v % 8) of the row's 128.
+  auto issue_w = [&](int c) {
+    if (c < n_chunks) {
+      const uint32_t dst0 = wring_s + (c % kWStages) * S::kWStageBytes;
 #pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t)
-#pragma unroll
-    for (int i = 0; i < kOutPerLane; ++i) acc[t][i] = 0.0f;
-
-  // Register staging of one k chunk: vector v = threadIdx.x + kThreads * n.
-  uint4 wreg[kWVec], xreg[kXVec];
-  auto load_chunk = [&](int k0) {
-#pragma unroll
-    for (int n = 0; n < kWVec; ++n) {
-      const int v = threadIdx.x + kThreads * n;
-      const int row = v >> 3, kk = (v & 7) * 8;
-      const uint16_t* src = row < kDcT ? p.w_dkv + (int64_t)row * p.d_model
-                                       : p.w_kr + (int64_t)(row - kDcT) * p.d_model;
-      wreg[n] = __ldg(reinterpret_cast<const uint4*>(src + k0 + kk));
+      for (int n = 0; n < S::kWCopies; ++n) {
+        const int v = threadIdx.x + kThreads * n;
+        const int row = v >> 3, kk = (v & 7) * 8;
+        const uint16_t* src = row < kDcT ? p.w_dkv + (int64_t)row * p.d_model
+                                         : p.w_kr + (int64_t)(row - kDcT) * p.d_model;
+        cp_async16(dst0 + (row * kWStride + kk) * 2, src + c * kKc + kk);
+      }
     }
+    cp_async_commit();  // one group per chunk index, empty past the end
+  };
+  // x chunk: vector v = threadIdx.x + kThreads * n is token v / 8, k (v % 8) * 8.
+  uint4 xreg[S::kXVec];
+  auto load_x = [&](int c) {
 #pragma unroll
-    for (int n = 0; n < kXVec; ++n) {
+    for (int n = 0; n < S::kXVec; ++n) {
       const int v = threadIdx.x + kThreads * n;
       const int t = v >> 3, kk = (v & 7) * 8;
       xreg[n] = tok0 + t < p.n_tok
-                    ? __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)(tok0 + t) * p.d_model + k0 + kk))
+                    ? __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)(tok0 + t) * p.d_model + c * kKc + kk))
                     : make_uint4(0, 0, 0, 0);
     }
   };
-  auto store_chunk = [&](float* buf) {
-    float* ws = buf;
-    float* xs = buf + kDrow * kStride;
+  auto store_x = [&](float* xs) {
 #pragma unroll
-    for (int n = 0; n < kWVec; ++n) {
-      const int v = threadIdx.x + kThreads * n;
-      const int row = v >> 3, kk = (v & 7) * 8;
-      float4 lo, hi;
-      bf16x8_to_f32(wreg[n], lo, hi);
-      *reinterpret_cast<float4*>(ws + row * kStride + kk) = lo;
-      *reinterpret_cast<float4*>(ws + row * kStride + kk + 4) = hi;
-    }
-#pragma unroll
-    for (int n = 0; n < kXVec; ++n) {
+    for (int n = 0; n < S::kXVec; ++n) {
       const int v = threadIdx.x + kThreads * n;
       const int t = v >> 3, kk = (v & 7) * 8;
-      float4 lo, hi;
-      bf16x8_to_f32(xreg[n], lo, hi);
-      *reinterpret_cast<float4*>(xs + t * kStride + kk) = make_float4(lo.w, lo.x, lo.y, lo.z);
-      *reinterpret_cast<float4*>(xs + t * kStride + kk + 4) = make_float4(hi.w, hi.x, hi.y, hi.z);
+      const uint4 u = xreg[n];
+      *reinterpret_cast<float4*>(xs + t * kXStride + kk) =
+          make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+      *reinterpret_cast<float4*>(xs + t * kXStride + kk + 4) =
+          make_float4(bf16lo_to_f32(u.z), bf16hi_to_f32(u.z), bf16lo_to_f32(u.w), bf16hi_to_f32(u.w));
     }
   };
 
-  const int n_chunks = p.d_model / kKc;
-  load_chunk(0);
-  store_chunk(smem_f);
-  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kWStages - 1; ++c) issue_w(c);
+  load_x(0);
+  store_x(xbuf);
+  if (n_chunks > 1) load_x(1);
   for (int c = 0; c < n_chunks; ++c) {
-    const float* ws = smem_f + (c & 1) * kBufFloats;
-    const float* xs = ws + kDrow * kStride;
-    if (c + 1 < n_chunks) load_chunk((c + 1) * kKc);
-#pragma unroll 2
-    for (int kk = 0; kk < kKc; kk += 4) fma_step(acc, ws, xs, lane, warp * kTokPerWarp, kk);
-    if (c + 1 < n_chunks) store_chunk(smem_f + ((c + 1) & 1) * kBufFloats);
-    __syncthreads();
-  }
-
-  // 3D rotary embedding of the rope dims: output d_c + lane is the lane's last output.
-  constexpr int kRope = kOutPerLane - 1;
-  {
-    const int pair = lane >> 1;
-    const bool even = (lane & 1) == 0;
-    const int per_frame = p.grid_h * p.grid_w;
-#pragma unroll
-    for (int t = 0; t < kTokPerWarp; ++t) {
-      const int tok = tok0 + warp * kTokPerWarp + t;
-      const float v = acc[t][kRope];
-      const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-      if (tok < p.n_tok) {
-        const int f = tok / per_frame;
-        const int rem = tok - f * per_frame;
-        const int row = rem / p.grid_w;
-        const int col = rem - row * p.grid_w;
-        float2 cs;
-        if (pair < kPairsT) cs = tab.t[f][pair];
-        else if (pair < kPairsT + kPairsH) cs = tab.h[row][pair - kPairsT];
-        else cs = tab.w[col][pair - kPairsT - kPairsH];
-        const float a = even ? v : other;
-        const float bb = even ? other : v;
-        acc[t][kRope] = even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
-                             : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
-      }
+    cp_async_wait<kWStages - 2>();  // this thread's copies of chunk c have landed
+    __syncthreads();                // everyone's have, and chunk c - 1 is consumed
+    issue_w(c + kWStages - 1);      // into the stage chunk c - 1 used
+    if (c + 1 < n_chunks) {
+      store_x(xbuf + ((c + 1) & 1) * S::kXBufFloats);
+      if (c + 2 < n_chunks) load_x(c + 2);
     }
+    compute(xbuf + (c & 1) * S::kXBufFloats, wring + (c % kWStages) * (S::kWStageBytes / 2));
   }
+  cp_async_wait<0>();
+}
 
-  // Stage the kTok x (d_c + 32) bf16 rows in shared memory, then write 16-byte vectors.
-  __syncthreads();
-  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_f);
-#pragma unroll
-  for (int t = 0; t < kTokPerWarp; ++t)
-#pragma unroll
-    for (int i = 0; i < kOutPerLane; ++i)
-      os[(warp * kTokPerWarp + t) * kDrow + lane + 32 * i] = __float2bfloat16_rn(acc[t][i]);
-  __syncthreads();
-  constexpr int kVecPerRow = kDrow * 2 / 16;
+// Rotates the rope value v of token `tok` (pair `pair`; `other` is the partner
+// lane's value, `even` whether this lane holds the pair's first dim).
+__device__ __forceinline__ float rope_rotate(const AppendParams& p, const RopeTable& tab, int tok, int pair,
+                                             bool even, float v, float other) {
+  const int per_frame = p.grid_h * p.grid_w;
+  const int f = tok / per_frame;
+  const int rem = tok - f * per_frame;
+  const int row = rem / p.grid_w;
+  const int col = rem - row * p.grid_w;
+  float2 cs;
+  if (pair < kPairsT) cs = tab.t[f][pair];
+  else if (pair < kPairsT + kPairsH) cs = tab.h[row][pair - kPairsT];
+  else cs = tab.w[col][pair - kPairsT - kPairsH];
+  const float a = even ? v : other;
+  const float bb = even ? other : v;
+  return even ? __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(bb, cs.y))
+              : __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(bb, cs.x));
+}
+
+// Writes the CTA's staged bf16 rows (kTok x kRow in shared memory) to their ring
+// slots as 16-byte vectors.
+template <int kRow, int kThreads>
+__device__ __forceinline__ void write_rows(const AppendParams& p, const __nv_bfloat16* os, int b, int tok0) {
+  constexpr int kVecPerRow = kRow * 2 / 16;
   for (int v = threadIdx.x; v < kTok * kVecPerRow; v += kThreads) {
     const int t = v / kVecPerRow, c = v - t * kVecPerRow;
     const int tok = tok0 + t;
     if (tok < p.n_tok) {
       const int64_t slot = (p.slot0 + tok) % p.cap;
-      uint4 val = *reinterpret_cast<const uint4*>(os + t * kDrow + c * 8);
-      *reinterpret_cast<uint4*>(p.cache + ((int64_t)b * p.cap + slot) * kDrow + c * 8) = val;
+      const uint4 val = *reinterpret_cast<const uint4*>(os + t * kRow + c * 8);
+      *reinterpret_cast<uint4*>(p.cache + ((int64_t)b * p.cap + slot) * kRow + c * 8) = val;
     }
   }
 }
 
+// ---- wide layout ------------------------------------------------------------
+//
+// Warp w owns tokens 4w .. 4w+3; lane l owns outputs l + 32 i, i < kN: kP content
+// pairs (l + 64 q, l + 64 q + 32) and the rope dim d_c + l.  k steps are 8 wide:
+// one 16-byte load per W row (8 bf16) and two per x row.  For a W load the 8
+// rows of a quarter-warp start 144 bytes apart (distinct 16-byte bank groups);
+// an x load is one address for the whole warp.
+template <int kDcT>
+struct Wide {
+  static constexpr int kRow = kDcT + kDr;
+  static constexpr int kN = kRow / 32;      // outputs per lane: 3, 5, 7, 9
+  static constexpr int kP = (kN - 1) / 2;   // content pairs per lane
+  static constexpr int kWarps = 8;
+  static constexpr int kT = kTok / kWarps;  // tokens per warp
+  static constexpr int kThreads = 32 * kWarps;
+  using S = Stage<kDcT, kThreads>;
+  static_assert(kDcT == 64 * kP, "kP content pairs + one rope dim per lane");
+
+  struct Frag {
+    uint4 w[kN];
+    float4 x[kT][2];
+  };
+
+  __device__ static __forceinline__ void load(Frag& f, const float* xs, const uint16_t* ws, int lane,
+                                              int tok_row0, int kk) {
+#pragma unroll
+    for (int i = 0; i < kN; ++i) f.w[i] = *reinterpret_cast<const uint4*>(ws + (lane + 32 * i) * kWStride + kk);
+#pragma unroll
+    for (int t = 0; t < kT; ++t)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        f.x[t][h] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kXStride + kk + 4 * h);
+  }
+
+  // One 8-wide k step on `cur`; the loads of the next step (k offset kk_next)
+  // into `nxt` are spread over it, about two per k.  Every accumulator takes
+  // k, k+1, ..., k+7 in turn (its sequential order).
+  __device__ static __forceinline__ void step(float2 (&acc2)[kT][kP], float (&acc1)[kT], const Frag& cur,
+                                              Frag& nxt, const float* xs, const uint16_t* ws, int lane,
+                                              int tok_row0, int kk_next) {
+    constexpr int kLoads = kN + 2 * kT;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+      for (int n = (kLoads * e) / 8; n < (kLoads * (e + 1)) / 8; ++n) {
+        if (n < kN) {
+          nxt.w[n] = *reinterpret_cast<const uint4*>(ws + (lane + 32 * n) * kWStride + kk_next);
+        } else {
+          const int t = (n - kN) >> 1, h = (n - kN) & 1;
+          nxt.x[t][h] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kXStride + kk_next + 4 * h);
+        }
+      }
+      float wf[kN];
+#pragma unroll
+      for (int i = 0; i < kN; ++i) wf[i] = widen(u4comp(cur.w[i], e >> 1), e);
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const float xv = f4comp(cur.x[t][e >> 2], e & 3);
+        const float2 xx = make_float2(xv, xv);
+#pragma unroll
+        for (int q = 0; q < kP; ++q)
+          acc2[t][q] = __ffma2_rn(xx, make_float2(wf[2 * q], wf[2 * q + 1]), acc2[t][q]);
+        acc1[t] = fmaf(xv, wf[kN - 1], acc1[t]);
+      }
+    }
+  }
+};
+
+template <int kDcT>
+__global__ void __launch_bounds__(Wide<kDcT>::kThreads, 1)
+    k_cache_append_wide(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
+  using L = Wide<kDcT>;
+  constexpr int kT = L::kT, kP = L::kP, kRow = L::kRow;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const int b = blockIdx.y;
+  const int tok0 = blockIdx.x * kTok;
+  const int lane = threadIdx.x & 31;
+  const int tok_row0 = (threadIdx.x >> 5) * kT;   // this warp's first token row (within the CTA)
+
+  float2 acc2[kT][kP];   // outputs (lane + 64 q, lane + 64 q + 32)
+  float acc1[kT];        // output d_c + lane (rope)
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+#pragma unroll
+    for (int q = 0; q < kP; ++q) acc2[t][q] = make_float2(0.0f, 0.0f);
+    acc1[t] = 0.0f;
+  }
+
+  run_chunks<kDcT, L::kThreads>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
+    // Steps in pairs (f0 -> f1 -> f0); the last step's prefetch reads the row
+    // padding at k offset 64 (in bounds, never used).
+    typename L::Frag f0, f1;
+    L::load(f0, xs, ws, lane, tok_row0, 0);
+#pragma unroll 2
+    for (int kk = 0; kk < kKc; kk += 16) {
+      L::step(acc2, acc1, f0, f1, xs, ws, lane, tok_row0, kk + 8);
+      L::step(acc2, acc1, f1, f0, xs, ws, lane, tok_row0, kk + 16);
+    }
+  });
+
+  // Rope: output d_c + lane is acc1; a pair (2p, 2p+1) sits in lanes (2p, 2p+1).
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+    const int tok = tok0 + tok_row0 + t;
+    const float other = __shfl_xor_sync(0xffffffffu, acc1[t], 1);
+    if (tok < p.n_tok) acc1[t] = rope_rotate(p, tab, tok, lane >> 1, (lane & 1) == 0, acc1[t], other);
+  }
+
+  __syncthreads();
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_raw);
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+    __nv_bfloat16* orow = os + (tok_row0 + t) * kRow;
+#pragma unroll
+    for (int q = 0; q < kP; ++q) {
+      orow[lane + 64 * q] = __float2bfloat16_rn(acc2[t][q].x);
+      orow[lane + 64 * q + 32] = __float2bfloat16_rn(acc2[t][q].y);
+    }
+    orow[kDcT + lane] = __float2bfloat16_rn(acc1[t]);
+  }
+  __syncthreads();
+  write_rows<kRow, L::kThreads>(p, os, b, tok0);
+}
+
+// ---- tall layout ------------------------------------------------------------
+//
+// Lane l = 8 g + j: token group g (0..3), output group j (0..7); warp q owns
+// output quarter q.  A thread holds tokens g + 4 t (t < 8) and outputs
+// q * 8 kN + j + 8 m (m < kN): pairs (m = 2r, 2r + 1) and a single m = kN - 1.
+// k steps are 4 wide: one 8-byte load per W row (4 bf16), one 16-byte load per
+// x row.  For a W load the 8 rows j of a half-warp start 144 bytes apart
+// (distinct bank pairs); an x load is one address per quarter-warp.
+template <int kDcT>
+struct Tall {
+  static constexpr int kRow = kDcT + kDr;
+  static constexpr int kN = kRow / 32;      // outputs per thread: 3, 5, 7, 9
+  static constexpr int kP = kN / 2;         // output pairs per thread
+  static constexpr int kT = 8;              // tokens per thread
+  static constexpr int kThreads = 128;
+  using S = Stage<kDcT, kThreads>;
+  static_assert(kN % 2 == 1, "kP pairs + one single output per thread");
+
+  struct Frag {
+    float4 x[kT];
+    uint2 w[kN];
+  };
+
+  __device__ static __forceinline__ void load(Frag& f, const float* xs, const uint16_t* ws, int x_row0,
+                                              int w_row0, int kk) {
+#pragma unroll
+    for (int m = 0; m < kN; ++m) f.w[m] = *reinterpret_cast<const uint2*>(ws + (w_row0 + 8 * m) * kWStride + kk);
+#pragma unroll
+    for (int t = 0; t < kT; ++t) f.x[t] = *reinterpret_cast<const float4*>(xs + (x_row0 + 4 * t) * kXStride + kk);
+  }
+
+  // One 4-wide k step on `cur`; the loads of the next step (k offset kk_next)
+  // into `nxt` are spread over it, a quarter before each k's FMAs.  Every
+  // accumulator takes k, k+1, k+2, k+3 in turn (its sequential order).
+  __device__ static __forceinline__ void step(float2 (&acc2)[kT][kP], float (&acc1)[kT], const Frag& cur,
+                                              Frag& nxt, const float* xs, const uint16_t* ws, int x_row0,
+                                              int w_row0, int kk_next) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+#pragma unroll
+      for (int m = e; m < kN; m += 4)
+        nxt.w[m] = *reinterpret_cast<const uint2*>(ws + (w_row0 + 8 * m) * kWStride + kk_next);
+#pragma unroll
+      for (int t = e; t < kT; t += 4)
+        nxt.x[t] = *reinterpret_cast<const float4*>(xs + (x_row0 + 4 * t) * kXStride + kk_next);
+      float wf[kN];
+#pragma unroll
+      for (int m = 0; m < kN; ++m) wf[m] = widen((e < 2) ? cur.w[m].x : cur.w[m].y, e);
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const float xv = f4comp(cur.x[t], e);
+        const float2 xx = make_float2(xv, xv);
+#pragma unroll
+        for (int r = 0; r < kP; ++r)
+          acc2[t][r] = __ffma2_rn(xx, make_float2(wf[2 * r], wf[2 * r + 1]), acc2[t][r]);
+        acc1[t] = fmaf(xv, wf[kN - 1], acc1[t]);
+      }
+    }
+  }
+};
+
+template <int kDcT>
+__global__ void __launch_bounds__(Tall<kDcT>::kThreads, 1)
+    k_cache_append_tall(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
+  using L = Tall<kDcT>;
+  constexpr int kT = L::kT, kN = L::kN, kP = L::kP, kRow = L::kRow;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const int b = blockIdx.y;
+  const int tok0 = blockIdx.x * kTok;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int j = lane & 7;
+  const int x_row0 = lane >> 3;               // first token row of this thread (within the CTA)
+  const int w_row0 = warp * 8 * kN + j;       // first output row of this thread
+
+  // Output m of token t: acc2[t][m / 2].x / .y for m < kN - 1, acc1[t] for m = kN - 1.
+  float2 acc2[kT][kP];
+  float acc1[kT];
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+#pragma unroll
+    for (int r = 0; r < kP; ++r) acc2[t][r] = make_float2(0.0f, 0.0f);
+    acc1[t] = 0.0f;
+  }
+  auto acc = [&](int t, int m) -> float& {
+    return m == kN - 1 ? acc1[t] : ((m & 1) ? acc2[t][m >> 1].y : acc2[t][m >> 1].x);
+  };
+
+  run_chunks<kDcT, L::kThreads>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
+    // Steps in pairs (f0 -> f1 -> f0); the last step's prefetch reads the row
+    // padding at k offset 64 (in bounds, never used).
+    typename L::Frag f0, f1;
+    L::load(f0, xs, ws, x_row0, w_row0, 0);
+#pragma unroll 2
+    for (int kk = 0; kk < kKc; kk += 8) {
+      L::step(acc2, acc1, f0, f1, xs, ws, x_row0, w_row0, kk + 4);
+      L::step(acc2, acc1, f1, f0, xs, ws, x_row0, w_row0, kk + 8);
+    }
+  });
+
+  // Rope: whether output w_row0 + 8 m is a rope dim is the same for the whole
+  // warp (d_c is a multiple of 8), and a pair (2p, 2p+1) sits in lanes j, j ^ 1.
+#pragma unroll
+  for (int m = 0; m < kN; ++m) {
+    const int o = w_row0 + 8 * m;
+    if (o - j < kDcT) continue;
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+      const int tok = tok0 + x_row0 + 4 * t;
+      const float other = __shfl_xor_sync(0xffffffffu, acc(t, m), 1);
+      if (tok < p.n_tok) acc(t, m) = rope_rotate(p, tab, tok, (o - kDcT) >> 1, (j & 1) == 0, acc(t, m), other);
+    }
+  }
+
+  __syncthreads();
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_raw);
+#pragma unroll
+  for (int t = 0; t < kT; ++t)
+#pragma unroll
+    for (int m = 0; m < kN; ++m) os[(x_row0 + 4 * t) * kRow + w_row0 + 8 * m] = __float2bfloat16_rn(acc(t, m));
+  __syncthreads();
+  write_rows<kRow, L::kThreads>(p, os, b, tok0);
+}
+
+// ---- launch -----------------------------------------------------------------
+
+template <class Kernel>
+cudaError_t smem_attr(Kernel k, int bytes, bool (&done)[64], int dev) {
+  if (dev < 0 || dev >= 64 || done[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+// The tall layout runs where two of its CTAs fit on an SM and there are more
+// tiles than SMs; everything else runs the wide layout.
 template <int kDcT>
 cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, cudaStream_t stream) {
-  using A = AppendCfg<kDcT>;
-  static bool attr_set[64] = {false};
+  using W = Wide<kDcT>;
+  using T = Tall<kDcT>;
+  static bool wide_attr[64] = {false}, tall_attr[64] = {false};
+  static int tall_fit[64] = {0};      // 0 unknown, else 1 + (two tall CTAs fit on an SM)
+  static int sm_count[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_cache_append<kDcT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         A::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  cudaError_t e = smem_attr(k_cache_append_wide<kDcT>, W::S::kSmemBytes, wide_attr, dev);
+  if (e == cudaSuccess) e = smem_attr(k_cache_append_tall<kDcT>, T::S::kSmemBytes, tall_attr, dev);
+  if (e != cudaSuccess) return e;
+  int sms = 148, fit2 = 0;
+  if (dev >= 0 && dev < 64) {
+    if (sm_count[dev] == 0) {
+      e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+    }
+    if (tall_fit[dev] == 0) {
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_cache_append_tall<kDcT>, T::kThreads,
+                                                        T::S::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      tall_fit[dev] = 1 + (per_sm >= 2);
+    }
+    sms = sm_count[dev];
+    fit2 = tall_fit[dev] - 1;
   }
   static thread_local RopeTable tab;
   const int per_frame = p.grid_h * p.grid_w;
   build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
-  dim3 grid((p.n_tok + A::kTok - 1) / A::kTok, batch);
-  k_cache_append<kDcT><<<grid, A::kThreads, A::kSmemBytes, stream>>>(p, tab);
+  dim3 grid((p.n_tok + kTok - 1) / kTok, batch);
+  if (fit2 && (int64_t)grid.x * grid.y > sms)
+    k_cache_append_tall<kDcT><<<grid, T::kThreads, T::S::kSmemBytes, stream>>>(p, tab);
+  else
+    k_cache_append_wide<kDcT><<<grid, W::kThreads, W::S::kSmemBytes, stream>>>(p, tab);
   return cudaGetLastError();
 }
 }  // namespace

@@ -74,3 +74,25 @@ def test_append_ragged_and_single_token(vm):
         got = to_bits(cache)
         assert np.array_equal(got[:, 3:3 + n_tok], ref)
         assert np.all(got[:, :3] == 0) and np.all(got[:, 3 + n_tok:] == 0)
+
+
+@pytest.mark.parametrize("d_c", [64, 128, 192, 256])
+def test_append_many_tiles_ragged(vm, d_c):
+    """More 32-token tiles than SMs (300 tiles: the layout with 8 tokens per thread
+    runs where two of its CTAs fit on an SM, d_c <= 192), a ragged last tile, a
+    ring that wraps, and a first frame t0 > 0."""
+    import torch
+    w = workload.CONFIGS["480p"].with_(d_c=d_c)
+    wts = workload.layer_weights(w)
+    batch, n_tok, cap, slot0, t0 = 2, 4790, 4803, 4000, 5
+    x = workload.normal_bf16(w.seed + 101, (3,), (batch, n_tok, w.d_model))
+    cache = torch.zeros(batch, cap, d_c + 32, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_cache_append_dc(to_dev(x), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, slot0, t0,
+                            w.grid_h, w.grid_w)
+    vm.vmla_get_device_status()
+    ref = oracle.cache_append(x, wts["w_dkv"], wts["w_kr"], t0, w.grid_h, w.grid_w)
+    got = to_bits(cache)
+    slots = (slot0 + np.arange(n_tok)) % cap
+    assert np.array_equal(got[:, slots], ref), f"d_c={d_c}: append not bit-exact"
+    untouched = np.setdiff1d(np.arange(cap), slots)
+    assert np.all(got[:, untouched] == 0)

@@ -117,6 +117,19 @@ def test_canary_latent_widths(vm, d_c):
     assert_guards(buf, f"chunk attention d_c={d_c}")
 
 
+@pytest.mark.parametrize("d_c", [128, 192])
+def test_canary_append_many_tiles(vm, d_c):
+    # 2 x 150 tiles of 32 tokens, the last one ragged: the layout with 8 tokens
+    # per thread, two CTAs per SM.
+    w = workload.CONFIGS["480p"].with_(d_c=d_c)
+    wts = workload.layer_weights(w)
+    x = to_dev(workload.normal_bf16(w.seed + 7, (5,), (2, 4790, w.d_model)))
+    cbuf, cache = guarded(2, 4790, d_c + 32)
+    vm.vmla_cache_append_dc(x, to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, 0, 0, w.grid_h, w.grid_w)
+    vm.vmla_get_device_status()
+    assert_guards(cbuf, f"append many tiles d_c={d_c}")
+
+
 def test_canary_projections(vm):
     # 189 tokens (a partial M tile), d_model 384: N = 384 + 96 for the query
     # projection (a part-filled rope half) and N = 384 for the output projection.
