@@ -96,3 +96,18 @@ def test_append_many_tiles_ragged(vm, d_c):
     assert np.array_equal(got[:, slots], ref), f"d_c={d_c}: append not bit-exact"
     untouched = np.setdiff1d(np.arange(cap), slots)
     assert np.all(got[:, untouched] == 0)
+
+
+@pytest.mark.parametrize("n_tok", [148 * 32, 148 * 32 + 1])
+def test_append_layout_switch(vm, n_tok):
+    """Either side of the layout switch on a 148-SM part: 148 tiles run the wide
+    layout, 149 (one token more) the tall one; both bit-exact."""
+    import torch
+    w = workload.CONFIGS["480p"]
+    wts = workload.layer_weights(w)
+    x = workload.normal_bf16(w.seed + 211, (n_tok,), (1, n_tok, w.d_model))
+    cache = torch.zeros(1, n_tok, 224, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_cache_append(to_dev(x), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, 0, 2, w.grid_h, w.grid_w)
+    vm.vmla_get_device_status()
+    ref = oracle.cache_append(x, wts["w_dkv"], wts["w_kr"], 2, w.grid_h, w.grid_w)
+    assert np.array_equal(to_bits(cache), ref)
