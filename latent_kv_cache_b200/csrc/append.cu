@@ -25,7 +25,9 @@
 //  - the FMAs of two outputs of a token are issued as one fma.rn.f32x2 (two
 //    separately rounded fp32 FMAs, the same bits as two fmaf), which frees the
 //    issue slots the widening costs;
-//  - x is widened to fp32 once per CTA when it is staged.
+//  - x is widened to fp32 once per CTA when it is staged, except in the wide
+//    layout at d_c >= 192, where it too stays bf16 and is widened per use (its
+//    loads then take half the shared-memory wavefronts).
 // Two thread layouts share this scheme:
 //  - wide (8 warps, two per scheduler): warp w owns tokens 4w .. 4w+3, lane l
 //    owns outputs l + 32 i.  Used when each SM holds one tile.
@@ -36,7 +38,7 @@
 //
 // Operands per 64-wide k chunk: W (d_c + 32 rows of bf16) is copied by
 // cp.async into a 3-stage ring; x (32 rows) is loaded one chunk ahead into
-// registers, widened and stored into a double buffer.  The k steps of a chunk
+// registers and stored (widened, or as bf16) into a double buffer.  The k steps of a chunk
 // are software pipelined: the loads of step s + 1 are spread over the FMAs of
 // step s.
 #include <cuda_bf16.h>
@@ -66,12 +68,13 @@ struct AppendParams {
   int grid_w;
 };
 
-// Shared-memory plan and staging shares of a layout with kThreads threads.
-template <int kDcT, int kThreads>
+// Shared-memory plan and staging shares of a layout with kThreads threads; with
+// kXRaw, x rows stay bf16 (kWStride elements per row).
+template <int kDcT, int kThreads, bool kXRaw = false>
 struct Stage {
   static constexpr int kRow = kDcT + kDr;                    // cached scalars per token
   static constexpr int kWStageBytes = kRow * kWStride * 2;
-  static constexpr int kXBufFloats = kTok * kXStride;
+  static constexpr int kXBufFloats = kXRaw ? kTok * kWStride / 2 : kTok * kXStride;
   static constexpr int kSmemBytes = kWStages * kWStageBytes + 2 * kXBufFloats * 4;
   static constexpr int kWCopies = kRow * (kKc / 8) / kThreads;  // 16-byte W copies per thread per chunk
   static constexpr int kXVec = kTok * (kKc / 8) / kThreads;     // 16-byte x loads per thread per chunk
@@ -102,10 +105,10 @@ __device__ __forceinline__ float widen(uint32_t word, int e) {
 // The chunk pipeline shared by both layouts: W ring by cp.async, x staged
 // through registers, one __syncthreads per chunk.  `compute(xs, ws)` runs the
 // FMAs of one chunk.
-template <int kDcT, int kThreads, class Compute>
+template <int kDcT, int kThreads, bool kXRaw, class Compute>
 __device__ __forceinline__ void run_chunks(const AppendParams& p, uint8_t* smem_raw, int b, int tok0,
                                            Compute&& compute) {
-  using S = Stage<kDcT, kThreads>;
+  using S = Stage<kDcT, kThreads, kXRaw>;
   uint16_t* wring = reinterpret_cast<uint16_t*>(smem_raw);
   float* xbuf = reinterpret_cast<float*>(smem_raw + kWStages * S::kWStageBytes);
   const uint32_t wring_s = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
@@ -146,6 +149,10 @@ __device__ __forceinline__ void run_chunks(const AppendParams& p, uint8_t* smem_
       const int v = threadIdx.x + kThreads * n;
       const int t = v >> 3, kk = (v & 7) * 8;
       const uint4 u = xreg[n];
+      if constexpr (kXRaw) {
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(xs) + t * kWStride + kk) = u;
+        continue;
+      }
       *reinterpret_cast<float4*>(xs + t * kXStride + kk) =
           make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
       *reinterpret_cast<float4*>(xs + t * kXStride + kk + 4) =
@@ -221,13 +228,36 @@ struct Wide {
   static constexpr int kWarps = 8;
   static constexpr int kT = kTok / kWarps;  // tokens per warp
   static constexpr int kThreads = 32 * kWarps;
-  using S = Stage<kDcT, kThreads>;
+  // x stays bf16 in shared memory (widened per use, like W) at d_c >= 192, where
+  // the halved x wavefronts pay for the widening; at d_c = 64 and 128 it is
+  // staged as fp32.
+  static constexpr bool kXRaw = kDcT >= 192;
+  using S = Stage<kDcT, kThreads, kXRaw>;
   static_assert(kDcT == 64 * kP, "kP content pairs + one rope dim per lane");
 
+  // x[t][h]: fp32 k + 4h .. k + 4h + 3 of token row tok_row0 + t, or (kXRaw)
+  // x[t][0] = 8 bf16 of that row.
   struct Frag {
     uint4 w[kN];
-    float4 x[kT][2];
+    float4 x[kT][kXRaw ? 1 : 2];
   };
+  static constexpr int kXLoads = kXRaw ? 1 : 2;   // x loads per token per step
+  __device__ static __forceinline__ float4 load_x(const float* xs, int row, int kk, int h) {
+    if constexpr (kXRaw) {
+      return *reinterpret_cast<const float4*>(reinterpret_cast<const uint16_t*>(xs) + row * kWStride + kk);
+    } else {
+      return *reinterpret_cast<const float4*>(xs + row * kXStride + kk + 4 * h);
+    }
+  }
+  // fp32 value of x at k offset e (0..7) of the step.
+  __device__ static __forceinline__ float x_at(const float4 (&x)[kXRaw ? 1 : 2], int e) {
+    if constexpr (kXRaw) {
+      const float4 v = x[0];
+      return widen(__float_as_uint(f4comp(v, e >> 1)), e);
+    } else {
+      return f4comp(x[e >> 2], e & 3);
+    }
+  }
 
   __device__ static __forceinline__ void load(Frag& f, const float* xs, const uint16_t* ws, int lane,
                                               int tok_row0, int kk) {
@@ -236,8 +266,7 @@ struct Wide {
 #pragma unroll
     for (int t = 0; t < kT; ++t)
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        f.x[t][h] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kXStride + kk + 4 * h);
+      for (int h = 0; h < kXLoads; ++h) f.x[t][h] = load_x(xs, tok_row0 + t, kk, h);
   }
 
   // One 8-wide k step on `cur`; the loads of the next step (k offset kk_next)
@@ -246,7 +275,7 @@ struct Wide {
   __device__ static __forceinline__ void step(float2 (&acc2)[kT][kP], float (&acc1)[kT], const Frag& cur,
                                               Frag& nxt, const float* xs, const uint16_t* ws, int lane,
                                               int tok_row0, int kk_next) {
-    constexpr int kLoads = kN + 2 * kT;
+    constexpr int kLoads = kN + kXLoads * kT;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
 #pragma unroll
@@ -254,8 +283,8 @@ struct Wide {
         if (n < kN) {
           nxt.w[n] = *reinterpret_cast<const uint4*>(ws + (lane + 32 * n) * kWStride + kk_next);
         } else {
-          const int t = (n - kN) >> 1, h = (n - kN) & 1;
-          nxt.x[t][h] = *reinterpret_cast<const float4*>(xs + (tok_row0 + t) * kXStride + kk_next + 4 * h);
+          const int t = (n - kN) / kXLoads, h = (n - kN) % kXLoads;
+          nxt.x[t][h] = load_x(xs, tok_row0 + t, kk_next, h);
         }
       }
       float wf[kN];
@@ -263,7 +292,7 @@ struct Wide {
       for (int i = 0; i < kN; ++i) wf[i] = widen(u4comp(cur.w[i], e >> 1), e);
 #pragma unroll
       for (int t = 0; t < kT; ++t) {
-        const float xv = f4comp(cur.x[t][e >> 2], e & 3);
+        const float xv = x_at(cur.x[t], e);
         const float2 xx = make_float2(xv, xv);
 #pragma unroll
         for (int q = 0; q < kP; ++q)
@@ -294,7 +323,7 @@ __global__ void __launch_bounds__(Wide<kDcT>::kThreads, 1)
     acc1[t] = 0.0f;
   }
 
-  run_chunks<kDcT, L::kThreads>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
+  run_chunks<kDcT, L::kThreads, L::kXRaw>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
     // Steps in pairs (f0 -> f1 -> f0); the last step's prefetch reads the row
     // padding at k offset 64 (in bounds, never used).
     typename L::Frag f0, f1;
@@ -418,7 +447,7 @@ __global__ void __launch_bounds__(Tall<kDcT>::kThreads, 1)
     return m == kN - 1 ? acc1[t] : ((m & 1) ? acc2[t][m >> 1].y : acc2[t][m >> 1].x);
   };
 
-  run_chunks<kDcT, L::kThreads>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
+  run_chunks<kDcT, L::kThreads, false>(p, smem_raw, b, tok0, [&](const float* xs, const uint16_t* ws) {
     // Steps in pairs (f0 -> f1 -> f0); the last step's prefetch reads the row
     // padding at k offset 64 (in bounds, never used).
     typename L::Frag f0, f1;
