@@ -1,0 +1,55 @@
+"""bench.py end to end on the GPU: the small workload's JSON line carries every
+key the measurement contract asks for, with values that make sense."""
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*args):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_bench_tiny_line():
+    b = _run("--workload", "tiny", "--steps", "3", "--warmup", "3", "--no-cpu-baseline")
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in b, k
+    assert b["n_gpus"] == 1 and b["steps"] == 3 and b["warmup"] == 3
+    assert b["value"] > 0 and b["ms_per_step"] > 0
+    assert b["config"]["workload"].startswith("tiny")
+    r = b["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] > 0
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert r["traffic"] is None            # the committed ncu summary covers the 480P workload only
+    e = b["e2e"]
+    assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert b["gpu_launches"] == 2 * b["steps"]
+    a = b["append"]
+    assert a["bound"] == "alu" and 0 < a["frac"] < 1.5
+    assert b["dense"]["ms"] > 0 and b["nonabsorbed"]["ms_total"] > 0
+    assert set(b["dc_sweep"]) == {"64", "128", "192", "256"}
+
+
+def test_bench_reference_arm_line():
+    b = _run("--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0")
+    assert b["impl"] == "reference"
+    assert b["value"] > 0 and b["cpu_baseline"]["kind"] == "oracle"
+    assert b["e2e"]["h2d_bytes_per_step"] == 0 and b["e2e"]["d2h_bytes_per_step"] == 0
+    assert b["e2e"]["value"] == b["value"] and b["e2e"]["unit"] == b["unit"]
