@@ -38,9 +38,9 @@
 //
 // Operands per 64-wide k chunk: W (d_c + 32 rows of bf16) is copied by
 // cp.async into a 3-stage ring; x (32 rows) is loaded one chunk ahead into
-// registers and stored (widened, or as bf16) into a double buffer.  The k steps of a chunk
-// are software pipelined: the loads of step s + 1 are spread over the FMAs of
-// step s.
+// registers and stored (widened, or as bf16) into a double buffer.  The k steps
+// of a chunk are software pipelined: the loads of step s + 1 are spread over the
+// FMAs of step s.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
