@@ -91,6 +91,15 @@ def test_chunk_attention_ragged_and_small(vm):
     assert_close(got, ref, "ragged")
 
 
+def test_chunk_attention_ragged_batch(vm):
+    # three samples (independent seeds) of the ragged shape: batch indexing of
+    # queries, cache rows and outputs with partial query and key tiles
+    w = workload.CONFIGS["tiny"].with_(grid_h=7, grid_w=9, cached_frames=4, heads=3, batch=3, seed=91)
+    got, ref = _mla_case(vm, w)
+    assert_close(got, ref, "ragged batch 3")
+    assert not np.allclose(got[0], got[1])
+
+
 def test_chunk_attention_poisoned_slots_ignored(vm):
     # slots past n_kv hold NaN; they must never reach the output
     got, ref = _mla_case(vm, workload.CONFIGS["tiny"], cap_extra=300, poison=True)
@@ -184,6 +193,12 @@ def test_dense_attention_tiny_full(vm):
 def test_dense_attention_ragged(vm):
     got, ref = _dense_case(vm, workload.CONFIGS["tiny"].with_(grid_h=7, grid_w=9, cached_frames=4, heads=3))
     assert_close(got, ref, "dense ragged")
+
+
+def test_dense_attention_ragged_batch(vm):
+    w = workload.CONFIGS["tiny"].with_(grid_h=7, grid_w=9, cached_frames=4, heads=3, batch=3, seed=92)
+    got, ref = _dense_case(vm, w)
+    assert_close(got, ref, "dense ragged batch 3")
 
 
 def test_dense_attention_480p_sampled(vm):

@@ -47,12 +47,14 @@ def test_materialize_kv_matches_definition(vm):
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3)
 
 
-@pytest.mark.parametrize("name", ["tiny", "ragged"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "ragged_batch"])
 def test_materialized_attention_full(vm, name):
     import torch
     w = workload.CONFIGS["tiny"]
     if name == "ragged":
         w = w.with_(grid_h=7, grid_w=9, cached_frames=4, heads=3)
+    if name == "ragged_batch":
+        w = w.with_(grid_h=7, grid_w=9, cached_frames=4, heads=3, batch=3, seed=93)
     wts, act, cache, ref_cache = _setup(vm, w, cap_extra=3)
     kv = torch.empty(w.batch, w.n_kv, 2 * w.heads, 128, dtype=torch.bfloat16, device="cuda")
     vm.vmla_materialize_kv(to_dev(wts["w_uk"]), to_dev(wts["w_uv"]), cache, w.n_kv, kv)
