@@ -35,6 +35,9 @@
 //    holds 8 tokens x (d_c + 32) / 32 outputs, half the operand words per FMA of
 //    the wide form.  With one warp per scheduler it stalls more, so it only wins
 //    where two tiles share an SM (more tiles than SMs, d_c <= 192).
+//  - slice (8 warps): for appends too small to fill the SMs, a CTA computes one
+//    64-output slice (or the rope slice) of a tile, so the tile's slices run on
+//    separate SMs.
 //
 // Operands per 64-wide k chunk: W (d_c + 32 rows of bf16) is copied by
 // cp.async into a 3-stage ring; x (32 rows) is loaded one chunk ahead into
@@ -483,6 +486,154 @@ __global__ void __launch_bounds__(Tall<kDcT>::kThreads, 1)
   write_rows<kRow, L::kThreads>(p, os, b, tok0);
 }
 
+// ---- slice layout -----------------------------------------------------------
+//
+// For appends too small to fill the SMs: the d_c + 32 outputs are cut into d_c/64
+// content slices of 64 rows and the 32-row rope slice, and a CTA computes one
+// slice for 32 tokens (grid z = slice), so a chunk of T tiles runs as
+// T (d_c/64 + 1) CTAs.  8 warps of 4 tokens; in a content slice lane l owns rows
+// s0 + l and s0 + 32 + l (one paired FMA), in the rope slice row d_c + l.  Both
+// W and x stay bf16 in shared memory and arrive by cp.async through a deep ring
+// (a stage is only 64 W rows + 32 x rows), since a slice's short k steps leave
+// little time to hide each load.  Same arithmetic order as the other layouts.
+template <int kDcT>
+struct Slice {
+  static constexpr int kRow = kDcT + kDr;
+  static constexpr int kParts = kDcT / 64 + 1;   // content slices + the rope slice
+  static constexpr int kWRows = 64;
+  static constexpr int kWarps = 8;
+  static constexpr int kT = kTok / kWarps;       // tokens per warp
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kStages = 8;
+  static constexpr int kStageBytes = (kWRows + kTok) * kWStride * 2;   // W rows, then x rows
+  static constexpr int kSmemBytes = kStages * kStageBytes;
+  static constexpr int kCopies = (kWRows + kTok) * (kKc / 8) / kThreads;  // 16-byte copies per thread per chunk
+  static_assert(((kWRows + kTok) * (kKc / 8)) % kThreads == 0, "staging");
+  static_assert(kTok * kWRows * 2 <= kSmemBytes && kSmemBytes <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+// One CTA of the slice layout; kRope: the rope slice (rows d_c .. d_c + 31).
+template <int kDcT, bool kRope>
+__device__ __forceinline__ void slice_body(const AppendParams& p, const RopeTable& tab, uint8_t* smem_raw) {
+  using L = Slice<kDcT>;
+  constexpr int kT = L::kT, kRow = L::kRow, kStages = L::kStages;
+  constexpr bool rope = kRope;
+  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+  const int b = blockIdx.y;
+  const int tok0 = blockIdx.x * kTok;
+  const int part = blockIdx.z;
+  const int s0 = part * 64;                       // first output row of the slice
+  constexpr int n_rows = kRope ? kDr : 64;
+  const int lane = threadIdx.x & 31;
+  const int tok_row0 = (threadIdx.x >> 5) * kT;
+  const uint16_t* xb = p.x + (int64_t)b * p.n_tok * p.d_model;
+  const int n_chunks = p.d_model / kKc;
+
+  // Chunk c -> stage c % kStages: copy v = threadIdx.x + kThreads n is row v / 8
+  // (W rows first, then the 32 x rows), bytes 16 (v % 8) of the row's 128.
+  auto issue = [&](int c) {
+    if (c < n_chunks) {
+      const uint32_t dst0 = ring_s + (c % kStages) * L::kStageBytes;
+#pragma unroll
+      for (int n = 0; n < L::kCopies; ++n) {
+        const int v = threadIdx.x + L::kThreads * n;
+        const int row = v >> 3, kk = (v & 7) * 8;
+        const uint32_t dst = dst0 + (row * kWStride + kk) * 2;
+        if (row < L::kWRows) {
+          if (row >= n_rows) continue;
+          const int grow = s0 + row;
+          const uint16_t* src = grow < kDcT ? p.w_dkv + (int64_t)grow * p.d_model
+                                            : p.w_kr + (int64_t)(grow - kDcT) * p.d_model;
+          cp_async16(dst, src + c * kKc + kk);
+        } else {
+          const int t = row - L::kWRows;
+          const bool valid = tok0 + t < p.n_tok;
+          cp_async16_zfill(dst, xb + (int64_t)(valid ? tok0 + t : 0) * p.d_model + c * kKc + kk, valid);
+        }
+      }
+    }
+    cp_async_commit();  // one group per chunk index, empty past the end
+  };
+
+  float2 acc[kT];   // content: rows (s0 + lane, s0 + 32 + lane); rope: .x is row d_c + lane
+#pragma unroll
+  for (int t = 0; t < kT; ++t) acc[t] = make_float2(0.0f, 0.0f);
+
+#pragma unroll
+  for (int c = 0; c < kStages - 1; ++c) issue(c);
+  for (int c = 0; c < n_chunks; ++c) {
+    cp_async_wait<kStages - 2>();  // this thread's copies of chunk c have landed
+    __syncthreads();                // everyone's have, and chunk c - 1 is consumed
+    issue(c + kStages - 1);         // into the stage chunk c - 1 used
+    const uint16_t* ws = reinterpret_cast<const uint16_t*>(smem_raw + (c % kStages) * L::kStageBytes);
+    const uint16_t* xr = ws + L::kWRows * kWStride;
+#pragma unroll 2
+    for (int kk = 0; kk < kKc; kk += 8) {
+      const uint4 w0 = *reinterpret_cast<const uint4*>(ws + lane * kWStride + kk);
+      const uint4 w1 = rope ? w0 : *reinterpret_cast<const uint4*>(ws + (32 + lane) * kWStride + kk);
+      uint4 xq[kT];
+#pragma unroll
+      for (int t = 0; t < kT; ++t) xq[t] = *reinterpret_cast<const uint4*>(xr + (tok_row0 + t) * kWStride + kk);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float wa = widen(u4comp(w0, e >> 1), e);
+        const float wb = widen(u4comp(w1, e >> 1), e);
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+          const float xv = widen(u4comp(xq[t], e >> 1), e);
+          if constexpr (kRope) acc[t].x = fmaf(xv, wa, acc[t].x);
+          else acc[t] = __ffma2_rn(make_float2(xv, xv), make_float2(wa, wb), acc[t]);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  if constexpr (kRope) {  // a pair (2p, 2p+1) of rope dims sits in lanes (2p, 2p+1)
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+      const int tok = tok0 + tok_row0 + t;
+      const float other = __shfl_xor_sync(0xffffffffu, acc[t].x, 1);
+      if (tok < p.n_tok) acc[t].x = rope_rotate(p, tab, tok, lane >> 1, (lane & 1) == 0, acc[t].x, other);
+    }
+  }
+
+  // Stage the kTok x n_rows slice in shared memory, then write 16-byte vectors
+  // to columns [s0, s0 + n_rows) of each ring slot.
+  __syncthreads();
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(smem_raw);
+#pragma unroll
+  for (int t = 0; t < kT; ++t) {
+    __nv_bfloat16* orow = os + (tok_row0 + t) * L::kWRows;
+    orow[lane] = __float2bfloat16_rn(acc[t].x);
+    if (!rope) orow[32 + lane] = __float2bfloat16_rn(acc[t].y);
+  }
+  __syncthreads();
+  const int vec_per_row = n_rows / 8;
+  for (int v = threadIdx.x; v < kTok * vec_per_row; v += L::kThreads) {
+    const int t = v / vec_per_row, c = v - t * vec_per_row;
+    const int tok = tok0 + t;
+    if (tok < p.n_tok) {
+      const int64_t slot = (p.slot0 + tok) % p.cap;
+      const uint4 val = *reinterpret_cast<const uint4*>(os + t * L::kWRows + c * 8);
+      *reinterpret_cast<uint4*>(p.cache + ((int64_t)b * p.cap + slot) * kRow + s0 + c * 8) = val;
+    }
+  }
+}
+
+template <int kDcT>
+__global__ void __launch_bounds__(Slice<kDcT>::kThreads, 1)
+    k_cache_append_slice(const __grid_constant__ AppendParams p, const __grid_constant__ RopeTable tab) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  if (blockIdx.z == Slice<kDcT>::kParts - 1) slice_body<kDcT, true>(p, tab, smem_raw);
+  else slice_body<kDcT, false>(p, tab, smem_raw);
+}
+
 // ---- launch -----------------------------------------------------------------
 
 template <class Kernel>
@@ -493,19 +644,22 @@ cudaError_t smem_attr(Kernel k, int bytes, bool (&done)[64], int dev) {
   return e;
 }
 
-// The tall layout runs where two of its CTAs fit on an SM and there are more
-// tiles than SMs; everything else runs the wide layout.
+// The slice layout runs where all slices of all tiles fit in one wave (at most
+// one CTA per SM); the tall layout where two of its CTAs fit on an SM and there
+// are more tiles than SMs; everything else runs the wide layout.
 template <int kDcT>
 cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, cudaStream_t stream) {
   using W = Wide<kDcT>;
   using T = Tall<kDcT>;
-  static bool wide_attr[64] = {false}, tall_attr[64] = {false};
+  using Sl = Slice<kDcT>;
+  static bool wide_attr[64] = {false}, tall_attr[64] = {false}, slice_attr[64] = {false};
   static int tall_fit[64] = {0};      // 0 unknown, else 1 + (two tall CTAs fit on an SM)
   static int sm_count[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t e = smem_attr(k_cache_append_wide<kDcT>, W::S::kSmemBytes, wide_attr, dev);
   if (e == cudaSuccess) e = smem_attr(k_cache_append_tall<kDcT>, T::S::kSmemBytes, tall_attr, dev);
+  if (e == cudaSuccess) e = smem_attr(k_cache_append_slice<kDcT>, Sl::kSmemBytes, slice_attr, dev);
   if (e != cudaSuccess) return e;
   int sms = 148, fit2 = 0;
   if (dev >= 0 && dev < 64) {
@@ -527,7 +681,10 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
   const int per_frame = p.grid_h * p.grid_w;
   build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
   dim3 grid((p.n_tok + kTok - 1) / kTok, batch);
-  if (fit2 && (int64_t)grid.x * grid.y > sms)
+  const int64_t tiles = (int64_t)grid.x * grid.y;
+  if (tiles * Sl::kParts <= sms)
+    k_cache_append_slice<kDcT><<<dim3(grid.x, grid.y, Sl::kParts), Sl::kThreads, Sl::kSmemBytes, stream>>>(p, tab);
+  else if (fit2 && tiles > sms)
     k_cache_append_tall<kDcT><<<grid, T::kThreads, T::S::kSmemBytes, stream>>>(p, tab);
   else
     k_cache_append_wide<kDcT><<<grid, W::kThreads, W::S::kSmemBytes, stream>>>(p, tab);
