@@ -644,9 +644,10 @@ cudaError_t smem_attr(Kernel k, int bytes, bool (&done)[64], int dev) {
   return e;
 }
 
-// The slice layout runs where all slices of all tiles fit in one wave (at most
-// one CTA per SM); the tall layout where two of its CTAs fit on an SM and there
-// are more tiles than SMs; everything else runs the wide layout.
+// The slice layout runs where all slices of all tiles fit in one wave: one CTA
+// per SM, or (d_c >= 128, where a wide CTA takes longer than two slice CTAs
+// sharing an SM) two per SM.  The tall layout runs where two of its CTAs fit on
+// an SM and there are more tiles than SMs; everything else runs the wide layout.
 template <int kDcT>
 cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, cudaStream_t stream) {
   using W = Wide<kDcT>;
@@ -654,6 +655,7 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
   using Sl = Slice<kDcT>;
   static bool wide_attr[64] = {false}, tall_attr[64] = {false}, slice_attr[64] = {false};
   static int tall_fit[64] = {0};      // 0 unknown, else 1 + (two tall CTAs fit on an SM)
+  static int slice_fit[64] = {0};     // the same for slice CTAs
   static int sm_count[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -661,7 +663,7 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
   if (e == cudaSuccess) e = smem_attr(k_cache_append_tall<kDcT>, T::S::kSmemBytes, tall_attr, dev);
   if (e == cudaSuccess) e = smem_attr(k_cache_append_slice<kDcT>, Sl::kSmemBytes, slice_attr, dev);
   if (e != cudaSuccess) return e;
-  int sms = 148, fit2 = 0;
+  int sms = 148, fit2 = 0, slice_fit2 = 0;
   if (dev >= 0 && dev < 64) {
     if (sm_count[dev] == 0) {
       e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -674,15 +676,24 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
       if (e != cudaSuccess) return e;
       tall_fit[dev] = 1 + (per_sm >= 2);
     }
+    if (slice_fit[dev] == 0) {
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_cache_append_slice<kDcT>, Sl::kThreads,
+                                                        Sl::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      slice_fit[dev] = 1 + (per_sm >= 2);
+    }
     sms = sm_count[dev];
     fit2 = tall_fit[dev] - 1;
+    slice_fit2 = slice_fit[dev] - 1;
   }
   static thread_local RopeTable tab;
   const int per_frame = p.grid_h * p.grid_w;
   build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
   dim3 grid((p.n_tok + kTok - 1) / kTok, batch);
   const int64_t tiles = (int64_t)grid.x * grid.y;
-  if (tiles * Sl::kParts <= sms)
+  const int64_t slices = tiles * Sl::kParts;
+  if (slices <= sms || (kDcT >= 128 && slice_fit2 && slices <= 2 * (int64_t)sms))
     k_cache_append_slice<kDcT><<<dim3(grid.x, grid.y, Sl::kParts), Sl::kThreads, Sl::kSmemBytes, stream>>>(p, tab);
   else if (fit2 && tiles > sms)
     k_cache_append_tall<kDcT><<<grid, T::kThreads, T::S::kSmemBytes, stream>>>(p, tab);
