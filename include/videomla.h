@@ -180,7 +180,8 @@ vmla_status vmla_output_projection(const uint16_t* o, const uint16_t* w_o, int32
  * materialisation can be shared by every denoising step of a chunk.
  *
  * vmla_materialized_kv_bytes -- bytes of the materialised buffer kv[batch, n_kv, 2*heads, 128]
- *   (bf16; heads [0, heads) hold K_h, heads [heads, 2*heads) hold V_h); 0 on bad sizes.
+ *   (bf16; heads [0, heads) hold K_h, heads [heads, 2*heads) hold V_h); 0 on bad sizes and
+ *   on sizes whose byte count does not fit in int64.
  *
  * vmla_materialize_kv -- writes kv (caller-owned, vmla_materialized_kv_bytes bytes) from
  *   cache rows [0, n_kv) of cache[batch, cap, 224] and w_uk, w_uv [heads*128, 192].

@@ -196,7 +196,12 @@ static vmla_status check_latent_attention(const char* who, int32_t batch, int32_
 
 int64_t vmla_materialized_kv_bytes(int32_t batch, int32_t heads, int64_t n_kv) {
   if (batch < 1 || heads < 1 || n_kv < 1) return 0;
-  return (int64_t)batch * n_kv * 2 * heads * vmla::kDh * 2;
+  // batch * heads * 512 < 2^31 * 2^31 * 2^9 does not fit either, so divide step by step.
+  const int64_t per_key = (int64_t)heads * 2 * vmla::kDh * 2;  // <= 2^31 * 512
+  if ((int64_t)batch > INT64_MAX / per_key) return 0;
+  const int64_t per_row = (int64_t)batch * per_key;
+  if (n_kv > INT64_MAX / per_row) return 0;
+  return n_kv * per_row;
 }
 
 vmla_status vmla_materialize_kv(const uint16_t* w_uk, const uint16_t* w_uv, const uint16_t* cache,
@@ -250,6 +255,8 @@ vmla_status vmla_chunk_attention_nonabsorbed(const uint16_t* q, const uint16_t* 
                                           grid_h, grid_w, scale);
   if (st != VMLA_OK) return st;
   const int64_t need = vmla_materialized_kv_bytes(batch, heads, n_kv);
+  if (need <= 0)
+    return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention_nonabsorbed: workspace size overflows int64");
   if (workspace_bytes < need)
     return fail(VMLA_ERR_INVALID_ARG, "chunk_attention_nonabsorbed: workspace of %lld bytes, need %lld",
                 (long long)workspace_bytes, (long long)need);

@@ -69,6 +69,9 @@ vmla_status vmla_chunk_attention_nonabsorbed_noalloc(const uint16_t* q, const ui
                                                      int32_t grid_h, int32_t grid_w, float scale, uint16_t* out,
                                                      void* stream) {
   const int64_t need = vmla_materialized_kv_bytes(batch, heads, n_kv);
+  if (need <= 0 && batch >= 1 && heads >= 1 && n_kv >= 1)  // sizes whose buffer overflows int64
+    return vmla::record_error(VMLA_ERR_UNSUPPORTED,
+                              "chunk_attention_nonabsorbed_noalloc: workspace size overflows int64");
   if (need <= 0) {
     // Bad sizes: the full validation (and its message) comes from the workspace form.
     return vmla_chunk_attention_nonabsorbed(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,

@@ -112,3 +112,19 @@ def test_binding_rejects_non_cuda_tensors(vm):
         vm.vmla_cache_append(x, torch.zeros(192, 64, dtype=torch.bfloat16),
                              torch.zeros(32, 64, dtype=torch.bfloat16),
                              torch.zeros(1, 8, 224, dtype=torch.bfloat16), 0, 0, 2, 2)
+
+
+def test_materialized_kv_bytes_overflow_is_rejected(vm):
+    # batch 65535 x 512 heads x (2^31 - 1) keys x 512 bytes does not fit in int64:
+    # the size query returns 0 and both non-absorbed forms refuse before any launch.
+    L = vm.lib
+    f = ctypes.c_float
+    big = (1 << 31) - 1
+    assert L.vmla_materialized_kv_bytes(65535, 512, big) == 0
+    assert L.vmla_materialized_kv_bytes(1, 12, 32760) == 32760 * 2 * 12 * 128 * 2
+    assert L.vmla_chunk_attention_nonabsorbed(A, A, A, A, A, 65535, 192, 512, big, big, 0, 8, 8, f(0.1), A,
+                                              1 << 62, A, None) == 2
+    assert "overflow" in vm.vmla_last_error()
+    assert L.vmla_chunk_attention_nonabsorbed_noalloc(A, A, A, A, A, 65535, 192, 512, big, big, 0, 8, 8, f(0.1),
+                                                      A, None) == 2
+    assert "overflow" in vm.vmla_last_error()
