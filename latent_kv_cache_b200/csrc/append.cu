@@ -493,9 +493,11 @@ __global__ void __launch_bounds__(Tall<kDcT>::kThreads, 1)
 // slice for 32 tokens (grid z = slice), so a chunk of T tiles runs as
 // T (d_c/64 + 1) CTAs.  8 warps of 4 tokens; in a content slice lane l owns rows
 // s0 + l and s0 + 32 + l (one paired FMA), in the rope slice row d_c + l.  Both
-// W and x stay bf16 in shared memory and arrive by cp.async through a deep ring
-// (a stage is only 64 W rows + 32 x rows), since a slice's short k steps leave
-// little time to hide each load.  Same arithmetic order as the other layouts.
+// W and x stay bf16 in shared memory and arrive by cp.async through an 8-stage
+// ring (a stage is only 64 W rows + 32 x rows).  A 3-stage ring timed the same,
+// so the depth is not what hides the loads; at 8 stages a CTA takes 110.6 KB, and
+// two of them still fit on an SM, which the launcher's two-per-SM rule checks
+// with the occupancy API.  Same arithmetic order as the other layouts.
 template <int kDcT>
 struct Slice {
   static constexpr int kRow = kDcT + kDr;

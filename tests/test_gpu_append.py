@@ -111,3 +111,28 @@ def test_append_layout_switch(vm, n_tok):
     vm.vmla_get_device_status()
     ref = oracle.cache_append(x, wts["w_dkv"], wts["w_kr"], 2, w.grid_h, w.grid_w)
     assert np.array_equal(to_bits(cache), ref)
+
+
+@pytest.mark.parametrize("d_c,n_tok", [(128, 2304), (128, 2300), (192, 2304), (192, 2300), (256, 1600),
+                                       (256, 1590)])
+def test_append_two_slice_ctas_per_sm(vm, d_c, n_tok):
+    """More slice CTAs than SMs but at most two per SM (d_c >= 128): the slice
+    layout with two CTAs sharing an SM.  72 tiles x 3 or 4 slices, or 50 x 5 at
+    d_c = 256 (148 < slices <= 296 on a 148-SM part), a ragged last tile, a ring
+    that wraps, t0 > 0; bit-exact, nothing outside the written slots touched."""
+    import torch
+    w = workload.CONFIGS["480p"].with_(d_c=d_c)
+    wts = workload.layer_weights(w)
+    cap, t0 = n_tok + 13, 4
+    slot0 = cap - 100
+    x = workload.normal_bf16(w.seed + 307, (n_tok, d_c), (1, n_tok, w.d_model))
+    cache = torch.zeros(1, cap, d_c + 32, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_cache_append_dc(to_dev(x), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, slot0, t0,
+                            w.grid_h, w.grid_w)
+    vm.vmla_get_device_status()
+    ref = oracle.cache_append(x, wts["w_dkv"], wts["w_kr"], t0, w.grid_h, w.grid_w)
+    got = to_bits(cache)
+    slots = (slot0 + np.arange(n_tok)) % cap
+    assert np.array_equal(got[:, slots], ref), f"d_c={d_c}, {n_tok} tokens: append not bit-exact"
+    untouched = np.setdiff1d(np.arange(cap), slots)
+    assert np.all(got[:, untouched] == 0)

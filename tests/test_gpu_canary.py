@@ -146,3 +146,15 @@ def test_canary_projections(vm):
     vm.vmla_output_projection(q, to_dev(iw["w_o"]), y)
     vm.vmla_get_device_status()
     assert_guards(ybuf, "output projection")
+
+
+@pytest.mark.parametrize("d_c,n_tok", [(128, 2300), (192, 2300), (256, 1590)])
+def test_canary_append_two_slice_ctas(vm, d_c, n_tok):
+    # the slice layout at two CTAs per SM, with a ragged last tile
+    w = workload.CONFIGS["480p"].with_(d_c=d_c)
+    wts = workload.layer_weights(w)
+    x = to_dev(workload.normal_bf16(w.seed + 9, (n_tok,), (1, n_tok, w.d_model)))
+    cbuf, cache = guarded(1, n_tok, d_c + 32)
+    vm.vmla_cache_append_dc(x, to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, 0, 3, w.grid_h, w.grid_w)
+    vm.vmla_get_device_status()
+    assert_guards(cbuf, f"append two slice CTAs per SM d_c={d_c}")
