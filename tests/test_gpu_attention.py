@@ -73,15 +73,62 @@ def test_chunk_attention_tiny_peaked(vm):
 
 
 def test_chunk_attention_tiny_very_peaked(vm):
-    # queries x8 (scores ~8x the workload's): the bf16 rounding of the absorbed
-    # query q.W_UK (relative 2^-9 per element) moves each score by ~2^-9 of its
-    # magnitude, and with a near one-hot softmax that shows up directly in the
-    # largest outputs.  Relative L2 keeps the 1e-2 bound; max-abs is held to 8e-2.
+    """Queries x8 (scores ~8x the workload's, a near one-hot softmax).  Relative L2
+    keeps the 1e-2 bound; max-abs is held to 8e-2.  Any form whose score product
+    takes a bf16 operand formed from the latent carries that operand's rounding
+    (2^-9 relative): the absorbed query q.W_UK here, the materialised key c.W_UK^T
+    in the non-absorbed form and in a dense cache of those keys.  The CPU tests of
+    tests/test_tolerance_reading.py show that this one rounding alone exceeds
+    3e-2 at x8; this test shows the same on the three kernels, and that the
+    latent kernel's error is no larger than the other two forms'."""
+    import torch
     from helpers import errors
-    got, ref = _mla_case(vm, workload.CONFIGS["tiny"], q_mult=8.0)
-    rel, mx = errors(got, ref)
-    assert np.all(np.isfinite(got))
-    assert rel <= 1e-2 and mx <= 8e-2, (rel, mx)
+    w = workload.CONFIGS["tiny"]
+    wts = workload.layer_weights(w)
+    act = workload.batch_activations(w)
+    q8 = workload.bf16_bits(workload.bf16_to_f32(act["q"]) * np.float32(8.0))
+    qr8 = workload.bf16_bits(workload.bf16_to_f32(act["q_rope"]) * np.float32(8.0))
+    qr0 = np.zeros_like(qr8)
+    cache = torch.zeros(w.batch, w.n_kv, 224, dtype=torch.bfloat16, device="cuda")
+    gpu_fill_window(vm, w, to_dev(act["x"]), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache)
+    ref_cache = oracle.cache_append(act["x"], wts["w_dkv"], wts["w_kr"], 0, w.grid_h, w.grid_w)
+    wuk, wuv = to_dev(wts["w_uk"]), to_dev(wts["w_uv"])
+    shape = (w.batch, w.n_q, w.heads, 128)
+    kv = torch.empty(w.batch, w.n_kv, 2 * w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    # Dense per-head cache holding the latent's keys and values rounded to bf16
+    # (the rope queries are zero in this comparison: the dense kernel has no rope key).
+    kv_bits = workload.bf16_bits(oracle.materialized_kv(wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv)
+                                 .astype(np.float32))
+    kd = to_dev(np.ascontiguousarray(kv_bits[:, :, :w.heads]))
+    vd = to_dev(np.ascontiguousarray(kv_bits[:, :, w.heads:]))
+    err = {}
+    for rope_name, qr_bits in (("rope", qr8), ("no rope", qr0)):
+        ref = oracle.chunk_attention(q8, qr_bits, wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv, w.chunk_t0,
+                                     w.grid_h, w.grid_w, SCALE)
+        q_d, qr_d = to_dev(q8), to_dev(qr_bits)
+        out_a = torch.empty(*shape, dtype=torch.bfloat16, device="cuda")
+        vm.vmla_chunk_attention(q_d, qr_d, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE, out_a)
+        out_m = torch.empty_like(out_a)
+        vm.vmla_materialize_kv(wuk, wuv, cache, w.n_kv, kv)
+        vm.vmla_chunk_attention_materialized(q_d, qr_d, kv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                             out_m)
+        outs = {"absorbed": out_a, "non-absorbed": out_m}
+        if rope_name == "no rope":
+            out_d = torch.empty_like(out_a)
+            vm.vmla_dense_attention(q_d, kd, vd, SCALE, out_d)
+            outs["dense bf16 K_h"] = out_d
+        vm.vmla_get_device_status()
+        for form, o in outs.items():
+            got = to_f64(o)
+            assert np.all(np.isfinite(got)), (rope_name, form)
+            err[(rope_name, form)] = errors(got, ref)
+    for key, (rel, mx) in err.items():
+        assert rel <= 1e-2 and mx <= 8e-2, (key, rel, mx)
+    for key in (("rope", "non-absorbed"), ("no rope", "non-absorbed"), ("no rope", "dense bf16 K_h")):
+        assert err[key][1] > 3e-2, ("the bf16-key forms share the x8 excess", key, err[key])
+    for r in ("rope", "no rope"):
+        others = max(v[1] for k, v in err.items() if k[0] == r and k[1] != "absorbed")
+        assert err[(r, "absorbed")][1] <= 1.25 * others, (r, err)
 
 
 def test_chunk_attention_ragged_and_small(vm):
