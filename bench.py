@@ -43,7 +43,7 @@ METRIC = "MLA chunk-attention TFLOP/s & ms/chunk (Wan-1.3B 480P shape); % BF16 p
 UNIT = "TFLOP/s"
 SCALE = 160 ** -0.5
 FLUSH_BYTES = 256 << 20
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "chunk_attn_480p_ncu.md")
+PROFILED_TRAFFIC = os.path.join(ROOT, "profiles", "chunk_attn_480p_traffic.json")
 ATTN_SOURCES = [os.path.join(ROOT, "latent_kv_cache_b200", "csrc", f)
                 for f in ("attention.cu", "sm100.cuh", "common.cuh")]
 
@@ -56,6 +56,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="480p", choices=sorted(workload.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chunk", action="store_true",
+                    help="skip the per-chunk schedule figures of the 480P run (30 layers x 4 steps)")
+    ap.add_argument("--chunk-replays", type=int, default=7, help="timed chunk replays per schedule")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -91,19 +94,15 @@ def attn_source_hash() -> str:
 
 
 def profiled_traffic(workload_name: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
-    or None if the summary is missing, covers another workload, or the kernel
-    source changed since."""
+    """DRAM bytes per launch of the attention kernel: a profiled constant (one ncu
+    capture, kept with the source hash it was taken at), or None if the record is
+    missing, covers another workload, or the kernel source changed since."""
     try:
-        vals = {}
-        with open(PROFILE_SUMMARY) as f:
-            for line in f:
-                if line.startswith("- ") and ":" in line:
-                    k, v = line[2:].split(":", 1)
-                    vals[k.strip()] = v.strip().strip("`")
-        if vals.get("source_sha256_16") != attn_source_hash() or vals.get("workload") != workload_name:
+        with open(PROFILED_TRAFFIC) as f:
+            rec = json.load(f)
+        if rec.get("source_sha256_16") != attn_source_hash() or rec.get("workload") != workload_name:
             return None
-        return int(vals["dram_bytes_per_launch"])
+        return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -569,6 +568,15 @@ def run_ours(args, w, rank, world, local_rank):
     e2e_total = max_over_ranks(e2e_start.elapsed_time(e2e_end), dist, dev)
     e2e_value = job_value(world, args.steps, flops_step, e2e_total)
 
+    # ---- the full per-chunk schedule of this shape (30 layers x 4 denoising steps +
+    # 30 appends, CUDA graphs) and a >= 2 s back-to-back attention loop
+    chunk = None
+    if w.name == "480p" and not args.no_chunk:
+        del dbuf, h_x, h_q, h_qr, h_out
+        torch.cuda.empty_cache()
+        chunk = chunk_schedule_figures(vm, workload.CONFIGS["480p_chunk"].with_(seed=wr.seed), dev, rank, dist,
+                                       args.chunk_replays, args.warmup, local_rank, full_layer=False)
+
     peak, peak_sust, hbm, peak_src = measured_peaks()
     achieved = w.attention_flops() / (attn_mean * 1e-3) / 1e12
     traffic = profiled_traffic(w.name)
@@ -592,6 +600,8 @@ def run_ours(args, w, rank, world, local_rank):
                   "cache_bytes_per_token": {"mla": 224 * 2, "dense": 3072 * 2}},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": "profiled constant (profiles/chunk_attn_480p_traffic.json), "
+                                       "null unless the kernel source hash matches",
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "kernel": "k_chunk_attn"},
         "attention_dram_read_gbs": (traffic / (attn_mean * 1e-3) / 1e9) if traffic else None,
@@ -607,6 +617,8 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": gpu_launches,
         "clocks": clocks,
     }
+    if chunk is not None:
+        line["chunk_480p"] = chunk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, act, wts, args.cpu_seconds)
     if rank == 0:
@@ -621,7 +633,8 @@ def run_ours(args, w, rank, world, local_rank):
 # The full per-chunk schedule: L layers x (1 append + S denoising-step attentions),
 # captured once as a CUDA graph and replayed (timing-only inputs drawn on device)
 # ---------------------------------------------------------------------------
-def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, full_layer=False, chunks=1):
+def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, nonabsorbed_reuse=False,
+                         full_layer=False, attention_only=False, chunks=1):
     """Per-layer caches (filled by appends over the cached frames), the chunk's
     tokens, per-(layer, step) queries and outputs.  Returns, for each of `chunks`
     consecutive chunks, a list of zero-argument launch closures in schedule order,
@@ -631,7 +644,13 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, ful
     full_layer: each (step, layer) also computes its queries from the hidden
     states (q, q_r = x W_Q^T, x W_QR^T) and projects the heads' output (o W_O^T).
     dense: the per-head baseline, whose per-layer append writes the chunk's
-    K = x W_K^T and V = x W_V^T (3072 scalars per token) into its ring."""
+    K = x W_K^T and V = x W_V^T (3072 scalars per token) into its ring.
+    nonabsorbed: each layer materialises its K_h / V_h once per chunk into a
+    buffer of its own, which the chunk's denoising steps reuse (one buffer per
+    layer live during the chunk).  nonabsorbed_reuse: every (step, layer)
+    materialises into one shared buffer right before its attention (one buffer
+    live in all).  attention_only: the latent attentions alone, no appends (the
+    caches keep their window), for a back-to-back attention loop."""
     import torch
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
@@ -669,6 +688,10 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, ful
         if nonabsorbed:  # this layer's materialised K/V, live for the chunk's denoising steps
             L["kv"] = torch.empty(w.batch, w.n_kv, 2 * H, w.d_head, dtype=torch.bfloat16, device=dev)
         layers.append(L)
+    if nonabsorbed_reuse:  # one materialised K/V buffer for every (step, layer)
+        shared_kv = torch.empty(w.batch, w.n_kv, 2 * H, w.d_head, dtype=torch.bfloat16, device=dev)
+        for L in layers:
+            L["kv"] = shared_kv
     del x_win
     x_heads = x_chunk.view(w.batch, w.n_q, H, w.d_head) if dense else None
 
@@ -685,12 +708,14 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, ful
                             ops.append(lambda L=L, wn=wn, dst=dst: vm.vmla_output_projection(x_heads, L[wn], dst))
                     ops.append(lambda L=L, s=s: vm.vmla_dense_attention(L["q"][s], L["k"], L["v"], SCALE, L["out"][s]))
                     continue
-                if s == 0:  # the chunk's latents enter the window's ring once per layer
+                if s == 0 and not attention_only:  # the chunk's latents enter the window's ring once per layer
                     ops.append(lambda L=L: vm.vmla_cache_append(x_chunk, L["wd"], L["wk"], L["cache"], slot, t0,
                                                                 w.grid_h, w.grid_w))
                     if nonabsorbed:
                         ops.append(lambda L=L: vm.vmla_materialize_kv(L["wuk"], L["wuv"], L["cache"], w.n_kv, L["kv"]))
-                if nonabsorbed:
+                if nonabsorbed_reuse:
+                    ops.append(lambda L=L: vm.vmla_materialize_kv(L["wuk"], L["wuv"], L["cache"], w.n_kv, L["kv"]))
+                if nonabsorbed or nonabsorbed_reuse:
                     ops.append(lambda L=L, s=s: vm.vmla_chunk_attention_materialized(
                         L["q"][s], L["qr"][s], L["kv"], L["cache"], w.n_kv, t0, w.grid_h, w.grid_w, SCALE,
                         L["out"][s]))
@@ -725,8 +750,102 @@ def capture_graph(ops):
     return graph
 
 
+def chunk_schedule_figures(vm, w, dev, rank, dist, replays, warmup, local_rank=0, full_layer=True,
+                           sustained_s=2.0):
+    """ms per chunk of the full per-chunk schedule (one replay of a captured graph =
+    one chunk) for the absorbed, both non-absorbed and the dense schedules, plus a
+    back-to-back loop of the latent attentions alone for at least `sustained_s`
+    seconds with the SM clock sampled during it."""
+    import torch
+
+    # One graph per ring position: chunk c replays graph c mod G, so consecutive
+    # chunks slide the window (each append evicts the oldest frames).
+    G = w.n_kv // w.n_q if w.n_kv % w.n_q == 0 else 1
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+
+    def timed(graphs, n):
+        for i in range(max(warmup, len(graphs))):
+            graphs[i % len(graphs)].replay()
+        sync_all()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+        ev[1].record()
+        sync_all()
+        return max_over_ranks(ev[0].elapsed_time(ev[1]) / n, dist, dev)
+
+    def measure(n=None, sampler=None, **kind):
+        op_lists, _ = build_chunk_schedule(vm, w, dev, seed=(2000 if kind.get("dense") else 1000) + rank,
+                                           chunks=G, **kind)
+        graphs = [capture_graph(ops) for ops in op_lists]
+        vm.vmla_get_device_status()
+        if sampler is not None:
+            sampler.start()
+        ms = timed(graphs, n or replays)
+        clocks = sampler.stop() if sampler is not None else None
+        vm.vmla_get_device_status()
+        del graphs, op_lists
+        torch.cuda.empty_cache()
+        return ms, clocks
+
+    ms_chunk, clocks = measure(sampler=ClockSampler(local_rank))
+    ms_nonabs, _ = measure(nonabsorbed=True)
+    ms_reuse, _ = measure(nonabsorbed_reuse=True)
+    ms_dense, _ = measure(dense=True)
+    ms_full = measure(full_layer=True)[0] if full_layer else None
+    kv_one = w.batch * w.n_kv * 2 * w.heads * w.d_head * 2
+    res = {
+        "workload": (f"{w.name}: {w.layers} layers x ({w.steps} chunk attentions) + {w.layers} cache appends "
+                     f"per chunk, 480P shapes (Nq={w.n_q}, n_kv={w.n_kv}), one CUDA graph replay per chunk"),
+        "window": (f"sliding: {G} graphs (one per ring position) replayed in rotation, each chunk's append "
+                   f"evicts the oldest {w.chunk_frames} frames"),
+        "l2": "inputs larger than L2 (per-layer caches, queries and outputs)",
+        "replays": replays,
+        "ms_per_chunk": ms_chunk, "clocks": clocks,
+        "tflops": (w.layers * w.steps * w.attention_flops() + w.layers * w.append_flops()) / (ms_chunk * 1e-3) / 1e12,
+        "nonabsorbed": {"ms_per_chunk": ms_nonabs, "transient_kv_bytes": w.layers * kv_one,
+                        "how": "each layer materialises K_h/V_h once per chunk into its own buffer; "
+                               "the chunk's denoising steps reuse it"},
+        "nonabsorbed_reuse": {"ms_per_chunk": ms_reuse, "transient_kv_bytes": kv_one,
+                              "how": "every (step, layer) materialises into one shared buffer before its attention"},
+        "dense": {"ms_per_chunk": ms_dense, "layers": w.layers, "steps": w.steps,
+                  "append": "K = x W_K^T and V = x W_V^T of the chunk written into the dense ring per layer",
+                  "kv_cache_bytes": {"mla": w.layers * w.batch * w.n_kv * 448,
+                                     "dense": w.layers * w.batch * w.n_kv * 6144}},
+    }
+    if full_layer:
+        res["full_layer"] = {"ms_per_chunk": ms_full,
+                             "step": "per (step, layer): q/q_r projection + chunk attention + output projection; "
+                                     "one append per layer",
+                             "projection_flops_per_chunk": w.layers * w.steps * w.io_projection_flops()}
+    if sustained_s > 0:
+        # Back-to-back latent attentions (30 layers x 4 steps per replay, no appends)
+        # for >= sustained_s seconds: the power-capped steady state of a rollout.
+        est_ms = ms_chunk * w.layers * w.steps / (w.layers * w.steps + w.layers)
+        n = max(replays, int(sustained_s * 1e3 / max(est_ms, 1e-3)) + 1)
+        ms_att, sclocks = measure(n=n, sampler=ClockSampler(local_rank, period_s=0.005), attention_only=True)
+        tf = w.layers * w.steps * w.attention_flops() / (ms_att * 1e-3) / 1e12
+        _, peak_sust, _, src = measured_peaks()
+        mhz = (sclocks or {}).get("sm_mhz")
+        res["sustained"] = {
+            "seconds": n * ms_att / 1e3, "replays": n, "launches": n * w.layers * w.steps,
+            "ms_per_attention": ms_att / (w.layers * w.steps), "attention_tflops": tf,
+            "peak_sustained": peak_sust, "frac_of_sustained": tf / peak_sust if peak_sust else None,
+            "peak_source": f"{src} bf16_tflops_sustained",
+            "tflops_per_sm_ghz": tf / (mhz / 1e3) if mhz else None,
+            "clocks": sclocks,
+            "how": "graph replays of the 120 chunk attentions of one chunk (30 layers x 4 steps), back to back",
+        }
+    return res
+
+
 def run_chunk_schedule(args, w, rank, world, local_rank):
-    """ms per chunk of the full schedule (one replay of the captured graph = one chunk)."""
+    """ms per chunk of the full schedule, as its own JSON line."""
     import torch
     import latent_kv_cache_b200 as vm
 
@@ -737,45 +856,8 @@ def run_chunk_schedule(args, w, rank, world, local_rank):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    # One graph per ring position: chunk c replays graph c mod G, so consecutive
-    # chunks slide the window (each append evicts the oldest frames).
-    G = w.n_kv // w.n_q if w.n_kv % w.n_q == 0 else 1
-
-    def timed(graphs, n):
-        for i in range(max(args.warmup, len(graphs))):
-            graphs[i % len(graphs)].replay()
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ev[0].record()
-        for i in range(n):
-            graphs[i % len(graphs)].replay()
-        ev[1].record()
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        return max_over_ranks(ev[0].elapsed_time(ev[1]) / n, dist, dev)
-
-    def measure(sampler=None, **kind):
-        op_lists, _ = build_chunk_schedule(vm, w, dev, seed=(2000 if kind.get("dense") else 1000) + rank,
-                                           chunks=G, **kind)
-        graphs = [capture_graph(ops) for ops in op_lists]
-        vm.vmla_get_device_status()
-        if sampler is not None:
-            sampler.start()
-        ms = timed(graphs, args.steps)
-        clocks = sampler.stop() if sampler is not None else None
-        vm.vmla_get_device_status()
-        del graphs, op_lists
-        torch.cuda.empty_cache()
-        return ms, clocks
-
-    ms_chunk, clocks = measure(ClockSampler(local_rank))
-    ms_nonabs, _ = measure(nonabsorbed=True)
-    ms_full, _ = measure(full_layer=True)
-    ms_dense, _ = measure(dense=True)
+    fig = chunk_schedule_figures(vm, w, dev, rank, dist, args.steps, args.warmup, local_rank)
+    ms_chunk = fig["ms_per_chunk"]
     flops = w.layers * w.steps * w.attention_flops() + w.layers * w.append_flops()
     value = job_value(world, 1, flops, ms_chunk)
     n_launch = w.layers * w.steps + w.layers  # the absorbed graph, whose time is `value`
@@ -785,20 +867,10 @@ def run_chunk_schedule(args, w, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_desc(w), step=f"one chunk: {w.layers} layers x ({w.steps} chunk attentions) "
                                                f"+ {w.layers} cache appends, one CUDA graph replay",
-                       window=f"sliding: {G} graphs (one per ring position) replayed in rotation, each "
-                              f"chunk's append evicts the oldest {w.chunk_frames} frames",
-                       l2="inputs larger than L2 (per-layer caches, queries and outputs)"),
-        "nonabsorbed": {"ms_per_chunk": ms_nonabs,
-                        "transient_kv_bytes": w.layers * w.batch * w.n_kv * 2 * w.heads * w.d_head * 2},
-        "full_layer": {"ms_per_chunk": ms_full,
-                       "step": "per (step, layer): q/q_r projection + chunk attention + output projection; "
-                               "one append per layer",
-                       "projection_flops_per_chunk": w.layers * w.steps * w.io_projection_flops()},
-        "dense": {"ms_per_chunk": ms_dense, "layers": w.layers, "steps": w.steps,
-                  "append": "K = x W_K^T and V = x W_V^T of the chunk written into the dense ring per layer",
-                  "kv_cache_bytes": {"mla": w.layers * w.batch * w.n_kv * 448,
-                                     "dense": w.layers * w.batch * w.n_kv * 6144}},
-        "gpu_launches": args.steps * n_launch, "clocks": clocks,
+                       window=fig["window"], l2=fig["l2"]),
+        "nonabsorbed": fig["nonabsorbed"], "nonabsorbed_reuse": fig["nonabsorbed_reuse"],
+        "full_layer": fig["full_layer"], "dense": fig["dense"], "sustained": fig.get("sustained"),
+        "gpu_launches": args.steps * n_launch, "clocks": fig["clocks"],
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
