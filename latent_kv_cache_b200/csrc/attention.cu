@@ -9,9 +9,10 @@
 //     out_h,i     = ( sum_j softmax_j(score) c_j ) W_UV_h^T,
 // so one CTA streams (d_c + 32)-wide cache rows [c ; k_r] and never materialises K or V.
 //
-// One CTA = one 128-query tile of one head of one sample; heads are the fastest
-// grid index so the 12 CTAs that read the same cache tiles run together and
-// share them through L2.  Warp roles (320 threads):
+// One CTA = one 128-query tile of one head of one sample; in the latent kernel heads
+// are the fastest grid index so the 12 CTAs that read the same cache tiles run
+// together and share them through L2 (the per-head dense and materialised kernels
+// put query tiles fastest instead).  Warp roles (320 threads):
 //   warp 0      TMA producer: prologue operands, then key tiles into a ring.
 //   warp 1      TMEM allocation and the single MMA-issuing thread.
 //   warps 2..9  two softmax warpgroups; a thread owns one query row (= TMEM
@@ -389,8 +390,13 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x % p.heads;
-  const int q0 = (blockIdx.x / p.heads) * kBM;
+  // Grid order.  Latent kernel: heads fastest, so the 12 head-CTAs of a query
+  // tile, which read the same cache tiles, run together.  Dense and materialised
+  // kernels: query tiles fastest, so the CTAs that run together share one head's
+  // key/value tiles and each head's keys and values cross HBM about once.
+  const int n_qt = (p.n_q + kBM - 1) / kBM;
+  const int h = kMla ? (int)(blockIdx.x % p.heads) : (int)(blockIdx.x / n_qt);
+  const int q0 = (kMla ? (int)(blockIdx.x / p.heads) : (int)(blockIdx.x % n_qt)) * kBM;
   const int b = blockIdx.y;
   const int n_tiles = p.n_kv_tiles;
 
