@@ -165,6 +165,41 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// Tile schedule shared by the three roles.  Tiles whose N extent is full come
+// first, then the last N column when it is partial (it issues narrower MMAs and
+// costs less); tile positions are dealt to the pairs in rounds, alternating the
+// direction every round, so that a pair that drew early in one round draws late
+// in the next and the cheap partial tiles of the last rounds land on the pairs
+// that have done the least.  Returns false once the pair has no i-th tile.
+struct TileRef {
+  int m0;      // first output row of the pair tile
+  int n0;      // first output column
+  int n;       // output columns of the tile (a multiple of 32, <= 256)
+};
+__device__ __forceinline__ bool tile_at(const GemmParams& p, int pair, int n_pairs, int i, TileRef& t) {
+  const int pos = i * n_pairs + ((i & 1) ? n_pairs - 1 - pair : pair);
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  if (pos >= n_tiles) return false;
+  const int n_total = p.n0 + p.n1;
+  const int full_n = n_total / kTileN;  // N tiles of the full width
+  int mt, nt;
+  if (pos < p.tiles_m * full_n) {
+    mt = pos / full_n;
+    nt = pos - mt * full_n;
+  } else {  // the partial last column (tiles_n == full_n + 1)
+    mt = pos - p.tiles_m * full_n;
+    nt = full_n;
+  }
+  t.m0 = mt * kTileM;
+  t.n0 = nt * kTileN;
+  t.n = min(kTileN, n_total - t.n0);
+  // Each CTA stages its n/2 B rows with one box from B0 or from B1: if N0 falls
+  // inside one CTA's half, run the tile at full width instead (rows past N0 + N1
+  // are zero-filled and their columns are not stored).
+  if (t.n < kTileN && t.n0 < p.n0 && p.n0 < t.n0 + t.n && p.n0 != t.n0 + t.n / 2) t.n = kTileN;
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_bf16_pair(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -177,7 +212,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // 0 = leader (issues the MMAs)
   const int pair = (int)cluster_id_x(), n_pairs = (int)cluster_count_x();
-  const int n_tiles = p.tiles_m * p.tiles_n;
   const int nk = p.k / kBK;
 
   if (threadIdx.x == 0) {
@@ -213,9 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) last_use[s] = -1;
       int g = 0;
       bool ok = true;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs) {
-        const int m0 = (t / p.tiles_n) * kTileM + kHalf * (int)rank;
-        const int nrow = (t % p.tiles_n) * kTileN + kHalf * (int)rank;  // this CTA's half of the N tile
+      TileRef tr;
+      for (int i = 0; ok && tile_at(p, pair, n_pairs, i, tr); ++i) {
+        const int m0 = tr.m0 + kHalf * (int)rank;
+        // B rows of the pair MMA are split in halves of tr.n / 2: CTA r stages rows
+        // [r n/2, r n/2 + n/2) of the tile (the box always moves 128 rows; rows past
+        // the half are not read, rows past the matrix are zero-filled).
+        const int nrow = tr.n0 + (tr.n / 2) * (int)rank;
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int st = g % kStages, use = g / kStages;
           if (use > 0 && !(ok = mbar_wait(gbar(bars, G_EMPTY0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer)))
@@ -242,11 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t kId = idesc_bf16_f32(kTileM, kTileN, false, false);
       const uint32_t peer = 1;
       int g = 0, i = 0;
       bool ok = true;
-      for (int t = pair; t < n_tiles && ok; t += n_pairs, ++i) {
+      TileRef tr;
+      for (; ok && tile_at(p, pair, n_pairs, i, tr); ++i) {
+        const uint32_t kId = idesc_bf16_f32(kTileM, tr.n, false, false);
         const int acc = i & 1, acc_use = i >> 1;
         if (acc_use > 0 &&
             !(ok = mbar_wait_cluster(gbar(bars, G_ACCE0 + acc), (acc_use - 1) & 1, ctl, kDevTimeoutMma)))
@@ -280,20 +319,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // Epilogue warps 2..5: TMEM lane quadrant = warp % 4, row = 32 * quadrant + lane.
     const int qd = warp & 3;
-    int i = 0;
-    for (int t = pair; t < n_tiles; t += n_pairs, ++i) {
+    TileRef tr;
+    for (int i = 0; tile_at(p, pair, n_pairs, i, tr); ++i) {
       const int acc = i & 1, acc_use = i >> 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(gbar(bars, G_ACCF0 + acc), acc_use & 1, ctl,
                                                         kDevTimeoutSoftmax));
       if (!ok) break;
       tc_fence_after();
-      const int row0 = (t / p.tiles_n) * kTileM + kHalf * (int)rank + qd * 32;  // this warp's first row
-      const int ncol0 = (t % p.tiles_n) * kTileN;
+      const int row0 = tr.m0 + kHalf * (int)rank + qd * 32;  // this warp's first row
+      const int ncol0 = tr.n0;
       const uint32_t t_row = tmem + (uint32_t)(acc * kTileN) + ((uint32_t)(qd * 32) << 16);
       uint8_t* stg = smem + kStg + (warp - 2) * kStgWarp;
       uint32_t v[32];
+      const int n_c = tr.n / 32;
 #pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
+      for (int c = 0; c < n_c; ++c) {
         tmem_ld32(t_row + 32 * c, v);
         tmem_ld_wait();
 #pragma unroll
@@ -305,9 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7]));
           *reinterpret_cast<uint4*>(stg + lane * kStgRow + (c & 1) * 64 + q4 * 16) = w;
         }
-        if (c & 1) {  // 64 columns of 32 rows staged: store them as whole lines
+        if ((c & 1) || c == n_c - 1) {  // 64 (or a last 32) columns of 32 rows staged: store whole lines
           __syncwarp();
-          const int col = ncol0 + 32 * (c - 1);  // a 64-column block never straddles N0 (a multiple of 128)
+          // A 64-column block never straddles N0 (a multiple of 128).  When the tile
+          // has an odd number of 32-column groups it ends at N0 + N1, so the stale
+          // second half of its last block fails the column check below.
+          const int col = ncol0 + 64 * (c >> 1);
           uint16_t* base_ptr = col < p.n0 ? p.c0 + col : p.c1 + (col - p.n0);
           const int64_t ld = col < p.n0 ? p.ldc0 : p.ldc1;
 #pragma unroll

@@ -79,6 +79,15 @@ def test_query_projection_ragged(vm):
     _qproj(vm, w)
 
 
+@pytest.mark.parametrize("heads", [5, 7])
+def test_query_projection_narrow_last_column(vm, heads):
+    # N = 160 * heads = 800 or 1120: the last 256-column tile holds 32 or 96
+    # columns, all of the rope half, and runs narrower MMAs (each CTA of the pair
+    # stages 16 or 48 B rows; 1 or 3 column groups of 32).
+    w = workload.CONFIGS["tiny"].with_(grid_h=10, grid_w=20, heads=heads, d_model=256)
+    _qproj(vm, w)
+
+
 def test_query_projection_480p_full(vm):
     _qproj(vm, workload.CONFIGS["480p"])
 
