@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--workload", default="480p", choices=sorted(workload.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chunk", action="store_true",
-                    help="skip the per-chunk schedule figures of the 480P run (30 layers x 4 steps)")
+                    help="skip the per-chunk schedule and the batch-8 / 1080P figures of the 480P run")
     ap.add_argument("--chunk-replays", type=int, default=7, help="timed chunk replays per schedule")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -571,7 +571,11 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- the full per-chunk schedule of this shape (30 layers x 4 denoising steps +
     # 30 appends, CUDA graphs) and a >= 2 s back-to-back attention loop
     chunk = None
+    others = None
     if w.name == "480p" and not args.no_chunk:
+        others = {name: single_layer_figures(vm, workload.CONFIGS[name], dev, dist, 5, 3, local_rank,
+                                             seed=7000 + rank)
+                  for name in ("480p_b8", "1080p")}
         del dbuf, h_x, h_q, h_qr, h_out
         torch.cuda.empty_cache()
         chunk = chunk_schedule_figures(vm, workload.CONFIGS["480p_chunk"].with_(seed=wr.seed), dev, rank, dist,
@@ -619,6 +623,8 @@ def run_ours(args, w, rank, world, local_rank):
     }
     if chunk is not None:
         line["chunk_480p"] = chunk
+    if others is not None:
+        line["other_workloads"] = others
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, act, wts, args.cpu_seconds)
     if rank == 0:
@@ -731,6 +737,86 @@ def build_chunk_schedule(vm, w, dev, seed=0, dense=False, nonabsorbed=False, non
         return ops
 
     return [chunk_ops(ci) for ci in range(chunks)], layers
+
+
+def single_layer_figures(vm, w, dev, dist, reps, warmup, local_rank=0, seed=0):
+    """Event-timed append, latent attention, non-absorbed form and dense baseline of
+    one layer of workload `w` (timing-only inputs drawn on the device from a seeded
+    generator; the parity tests cover these shapes with the oracle's inputs).  L2 is
+    flushed before every timed call; clocks are sampled during the timed calls."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    D, H = w.d_model, w.heads
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    wd, wk = rnd(w.d_c, D, std=D ** -0.5), rnd(w.d_r, D, std=D ** -0.5)
+    wuk, wuv = rnd(H * w.d_head, w.d_c, std=w.d_c ** -0.5), rnd(H * w.d_head, w.d_c, std=w.d_c ** -0.5)
+    cache = torch.empty(w.batch, w.n_kv, w.d_c + w.d_r, dtype=torch.bfloat16, device=dev)
+    per = w.tokens_per_frame
+    for f0 in range(0, w.cached_frames, w.chunk_frames):
+        nf = min(w.chunk_frames, w.cached_frames - f0)
+        vm.vmla_cache_append(rnd(w.batch, nf * per, D), wd, wk, cache, f0 * per, f0, w.grid_h, w.grid_w)
+    x_chunk = rnd(w.batch, w.n_q, D)
+    q, qr = rnd(w.batch, w.n_q, H, w.d_head), rnd(w.batch, w.n_q, H, w.d_r)
+    out = torch.empty_like(q)
+    kd, vd = rnd(w.batch, w.n_kv, H, w.d_head), rnd(w.batch, w.n_kv, H, w.d_head)
+    kvm = torch.empty(w.batch, w.n_kv, 2 * H, w.d_head, dtype=torch.bfloat16, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    calls = {
+        "append": lambda: vm.vmla_cache_append(x_chunk, wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w),
+        "attention": lambda: vm.vmla_chunk_attention(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h,
+                                                     w.grid_w, SCALE, out),
+        "materialize": lambda: vm.vmla_materialize_kv(wuk, wuv, cache, w.n_kv, kvm),
+        "attention_materialized": lambda: vm.vmla_chunk_attention_materialized(
+            q, qr, kvm, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE, out),
+        "dense": lambda: vm.vmla_dense_attention(q, kd, vd, SCALE, out),
+    }
+    ms = {}
+    sampler = ClockSampler(local_rank)
+    for name, fn in calls.items():
+        for _ in range(warmup):
+            flush_w.zero_()
+            flush_r.max()
+            fn()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        if name == "attention":
+            sampler.start()
+        for e in ev:
+            flush_w.zero_()
+            flush_r.max()
+            e[0].record()
+            fn()
+            e[1].record()
+        torch.cuda.synchronize()
+        if name == "attention":
+            clocks = sampler.stop()
+        if dist is not None:
+            dist.barrier()
+        ms[name] = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / reps, dist, dev)
+    vm.vmla_get_device_status()
+    res = {
+        "workload": (f"{w.name}: B={w.batch}, {w.grid_h}x{w.grid_w} patches/frame, Nq={w.n_q}, n_kv={w.n_kv}, "
+                     f"H={H}x{w.d_head}, d_c={w.d_c}, d_r={w.d_r}"),
+        "reps": reps,
+        "attention": {"ms": ms["attention"], "tflops": w.attention_flops() / (ms["attention"] * 1e-3) / 1e12},
+        "append": {"us": ms["append"] * 1e3},
+        "nonabsorbed": {"ms_materialize": ms["materialize"], "ms_attention": ms["attention_materialized"],
+                        "ms_total": ms["materialize"] + ms["attention_materialized"],
+                        "attention_tflops": w.nonabsorbed_flops() / (ms["attention_materialized"] * 1e-3) / 1e12},
+        "dense": {"ms": ms["dense"], "tflops": w.dense_flops() / (ms["dense"] * 1e-3) / 1e12},
+        "clocks_attention": clocks,
+        "inputs": "drawn on the device (torch normal, seeded); timing only",
+    }
+    del cache, q, qr, out, kd, vd, kvm, flush_w, flush_r
+    torch.cuda.empty_cache()
+    return res
 
 
 def capture_graph(ops):

@@ -690,8 +690,9 @@ cudaError_t launch_cache_append_t(const AppendParams& p, int batch, int64_t t0, 
     slice_fit2 = slice_fit[dev] - 1;
   }
   static thread_local RopeTable tab;
+  static thread_local RopeTableKey tab_key;
   const int per_frame = p.grid_h * p.grid_w;
-  build_rope_table(&tab, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
+  build_rope_table(&tab, &tab_key, t0, (p.n_tok + per_frame - 1) / per_frame, p.grid_h, p.grid_w);
   dim3 grid((p.n_tok + kTok - 1) / kTok, batch);
   const int64_t tiles = (int64_t)grid.x * grid.y;
   const int64_t slices = tiles * Sl::kParts;

@@ -850,8 +850,9 @@ cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, 
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   static thread_local RopeTable tab;
+  static thread_local RopeTableKey tab_key;
   const int per_frame = grid_h * grid_w;
-  build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
+  build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
   k_chunk_attn<kDcT><<<grid, kThreads, L::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
@@ -943,8 +944,9 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   static thread_local RopeTable tab;
+  static thread_local RopeTableKey tab_key;
   const int per_frame = grid_h * grid_w;
-  build_rope_table(&tab, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
+  build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
   k_mat_attn<<<grid, kThreads, Layout<kKindMat>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();

@@ -23,10 +23,20 @@ struct RopeTable {
   float2 w[kMaxSide][kPairsW];
 };
 
-// Host: fill the table for frames [t0, t0 + n_frames), rows [0, grid_h), cols [0, grid_w).
+// What a host-side RopeTable currently holds (so that a call site can keep one
+// table and refill only the parts whose positions changed).
+struct RopeTableKey {
+  int64_t t0 = -1;
+  int n_frames = 0;
+  int grid_h = 0, grid_w = 0;
+};
+
+// Host: make `tab` hold frames [t0, t0 + n_frames), rows [0, grid_h), cols [0, grid_w).
 // Angles are computed in fp64 (pos * theta^(-2 i / d_axis)), then cos/sin in fp64
-// and rounded to fp32.
-void build_rope_table(RopeTable* tab, int64_t t0, int n_frames, int grid_h, int grid_w);
+// and rounded to fp32.  `key` records what the table holds; entries that already
+// hold the requested positions are not recomputed (a chunk's layers and denoising
+// steps share t0 and the grid, and a rollout keeps its grid).
+void build_rope_table(RopeTable* tab, RopeTableKey* key, int64_t t0, int n_frames, int grid_h, int grid_w);
 
 // Device-side status word of the current device (lazily looked up, cached per device).
 int* device_status_word();

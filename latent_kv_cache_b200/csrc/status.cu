@@ -24,28 +24,41 @@ int* device_status_word() {
   return cached[dev];
 }
 
-void build_rope_table(RopeTable* tab, int64_t t0, int n_frames, int grid_h, int grid_w) {
+void build_rope_table(RopeTable* tab, RopeTableKey* key, int64_t t0, int n_frames, int grid_h, int grid_w) {
   const int split[3] = {2 * kPairsT, 2 * kPairsH, 2 * kPairsW};
-  for (int f = 0; f < n_frames && f < kMaxFrames; ++f) {
-    for (int i = 0; i < kPairsT; ++i) {
-      double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[0]);
-      double a = (double)(t0 + f) * freq;
-      tab->t[f][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+  n_frames = n_frames < kMaxFrames ? n_frames : kMaxFrames;
+  grid_h = grid_h < kMaxSide ? grid_h : kMaxSide;
+  grid_w = grid_w < kMaxSide ? grid_w : kMaxSide;
+  if (key->t0 != t0 || key->n_frames < n_frames) {
+    for (int f = 0; f < n_frames; ++f) {
+      for (int i = 0; i < kPairsT; ++i) {
+        double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[0]);
+        double a = (double)(t0 + f) * freq;
+        tab->t[f][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
     }
+    key->t0 = t0;
+    key->n_frames = n_frames;
   }
-  for (int r = 0; r < grid_h && r < kMaxSide; ++r) {
-    for (int i = 0; i < kPairsH; ++i) {
-      double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[1]);
-      double a = (double)r * freq;
-      tab->h[r][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+  if (key->grid_h < grid_h) {  // rows [0, key->grid_h) already hold their values
+    for (int r = key->grid_h; r < grid_h; ++r) {
+      for (int i = 0; i < kPairsH; ++i) {
+        double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[1]);
+        double a = (double)r * freq;
+        tab->h[r][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
     }
+    key->grid_h = grid_h;
   }
-  for (int c = 0; c < grid_w && c < kMaxSide; ++c) {
-    for (int i = 0; i < kPairsW; ++i) {
-      double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[2]);
-      double a = (double)c * freq;
-      tab->w[c][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+  if (key->grid_w < grid_w) {
+    for (int c = key->grid_w; c < grid_w; ++c) {
+      for (int i = 0; i < kPairsW; ++i) {
+        double freq = std::pow(kRopeTheta, -2.0 * (double)i / (double)split[2]);
+        double a = (double)c * freq;
+        tab->w[c][i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
     }
+    key->grid_w = grid_w;
   }
 }
 
