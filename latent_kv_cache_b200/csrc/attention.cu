@@ -73,6 +73,12 @@ struct Cfg<kKindMla, kDcT> {
   static constexpr uint32_t kQaBytes = kStage;                   // Qa tile, same block structure
   static constexpr int kOCols = kDcT;
   static constexpr uint32_t kTmemS0 = 256, kTmemS1 = 384;
+  // With only two stages (d_c = 256) each stage is filled and released in two
+  // parts: X = content blocks [0, d_c/128) + the rope block, Y = the other content
+  // blocks.  P.C then runs as two N = d_c/2 halves, and X is refilled while the
+  // second half runs; the next score tile starts on X and waits for Y last.
+  static constexpr int kParts = kStages == 2 ? 2 : 1;
+  static constexpr int kNbX = kParts == 2 ? kNb / 2 : kNb;  // content blocks in part X
 };
 
 // Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
@@ -85,6 +91,7 @@ struct Cfg<kKindDense, kDcT> {
   static constexpr uint32_t kQaBytes = 0;
   static constexpr int kOCols = kDh;
   static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
+  static constexpr int kParts = 1;
 };
 
 // Materialised keys/values: Q = [q_h ; RoPE(q_r)] (80 cells) in TMEM; key tile =
@@ -98,6 +105,7 @@ struct Cfg<kKindMat, kDcT> {
   static constexpr uint32_t kQaBytes = 0;
   static constexpr int kOCols = kDh;
   static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
+  static constexpr int kParts = 1;
 };
 
 constexpr uint32_t kBlk128 = 128 * 128;  // 128 rows x 128 B: prologue / epilogue operand blocks
@@ -113,7 +121,7 @@ struct Layout {
   static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
   static constexpr uint32_t kMaxPad = kBytes - kUsed;  // alignment slack the kernel checks for
   static_assert(kUsed + 512 <= 232448, "shared memory (with at least 512 B of alignment slack)");
-  static_assert(C::kStages <= 8, "barrier slots");
+  static_assert(C::kStages * C::kParts <= 8, "barrier slots");
 };
 // The MLA prologue parks q (2 blocks) and W_UK_h (d_c/64 blocks) in ring stages
 // 0-1; the epilogue's W_UV_h (d_c/64 blocks) is one ring item.
@@ -127,8 +135,8 @@ static_assert(mla_fits<64>() && mla_fits<128>() && mla_fits<192>() && mla_fits<2
 
 enum Bar {
   B_PRO = 0, B_QABS, B_QA,
-  B_KVF0,                   // kStages "full" barriers
-  B_KVE0 = B_KVF0 + 8,      // kStages "empty" barriers
+  B_KVF0,                   // kStages "full" barriers per stage part
+  B_KVE0 = B_KVF0 + 8,      // kStages "empty" barriers per stage part
   B_SF0 = B_KVE0 + 8, B_SF1,
   B_PF0, B_PF1,
   B_PV, B_OA, B_OUT, B_DRAIN,
@@ -404,7 +412,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     mbar_init(bar_addr(bars, B_PRO), 1);
     mbar_init(bar_addr(bars, B_QABS), 1);
     mbar_init(bar_addr(bars, B_QA), kSoftmaxThreads);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStages * C::kParts; ++s) {  // part x of stage st: slot x * kStages + st
       mbar_init(bar_addr(bars, B_KVF0 + s), 1);
       mbar_init(bar_addr(bars, B_KVE0 + s), 1);
     }
@@ -433,9 +441,12 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------- producer -------------------------------
-      int last_use[kStages];
+      constexpr int kParts = C::kParts;
+      int last_use[kParts][kStages];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last_use[s] = -1;
+      for (int x = 0; x < kParts; ++x)
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) last_use[x][s] = -1;
       bool ok = true;
       if constexpr (kMla) {
         tma_prefetch_desc(&maps.q);
@@ -457,45 +468,45 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       }
       // MLA: n_tiles key tiles, then the W_UV_h blocks as one more ring item.
       const int n_items = kMla ? n_tiles + 1 : n_tiles;
-      for (int i = 0; i < n_items; ++i) {
+      for (int i = 0; ok && i < n_items; ++i) {
         const int st = i % kStages, use = i / kStages;
         const uint32_t sa = st0 + st * kStage;
-        if (use == 0) {
-          if (kMla && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
-        } else {
-          ok = mbar_wait(bar_addr(bars, B_KVE0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer);
-        }
-        if (!ok) break;
-        const uint32_t fb = bar_addr(bars, B_KVF0 + st);
-        const int kv0 = i * kBN;
-        if constexpr (kMla) {
-          if (i < n_tiles) {
-            mbar_arrive_expect_tx(fb, kStage);
-#pragma unroll
-            for (int blk = 0; blk < C::kNb; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
-            tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
+        if (use == 0 && kMla && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
+        for (int x = 0; ok && x < kParts; ++x) {
+          if (use > 0) ok = mbar_wait(bar_addr(bars, B_KVE0 + x * kStages + st), (use - 1) & 1, ctl,
+                                      kDevTimeoutProducer);
+          if (!ok) break;
+          const uint32_t fb = bar_addr(bars, B_KVF0 + x * kStages + st);
+          const int kv0 = i * kBN;
+          if constexpr (kMla) {
+            const int blo = x == 0 ? 0 : C::kNbX, bhi = x == 0 ? C::kNbX : C::kNb;
+            if (i < n_tiles) {
+              mbar_arrive_expect_tx(fb, (bhi - blo) * C::kBlkRows + (x == 0 ? 128u * 64u : 0u));
+              for (int blk = blo; blk < bhi; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
+              if (x == 0) tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
+            } else {
+              mbar_arrive_expect_tx(fb, (bhi - blo) * kBlk128);
+              for (int blk = blo; blk < bhi; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
+            }
           } else {
-            mbar_arrive_expect_tx(fb, C::kNb * kBlk128);
-#pragma unroll
-            for (int blk = 0; blk < C::kNb; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
+            const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
+            mbar_arrive_expect_tx(fb, kStage);
+            tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
+            tma_load_4d(sa + C::kBlkRows, &maps.k, fb, 64, h, kv0, b);
+            tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, hv, kv0, b);
+            tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, hv, kv0, b);
+            if constexpr (kMat) tma_load_3d(sa + 4 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
           }
-        } else {
-          const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
-          mbar_arrive_expect_tx(fb, kStage);
-          tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
-          tma_load_4d(sa + C::kBlkRows, &maps.k, fb, 64, h, kv0, b);
-          tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, hv, kv0, b);
-          tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, hv, kv0, b);
-          if constexpr (kMat) tma_load_3d(sa + 4 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
+          last_use[x][st] = use;
         }
-        last_use[st] = use;
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits.
         if (kMla) drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
-        for (int s = 0; s < kStages; ++s)
-          if (last_use[s] >= 0)
-            drain_wait(bar_addr(bars, B_KVF0 + s), last_use[s] & 1, p.wait_limit_ns, p.status);
+        for (int x = 0; x < kParts; ++x)
+          for (int s = 0; s < kStages; ++s)
+            if (last_use[x][s] >= 0)
+              drain_wait(bar_addr(bars, B_KVF0 + x * kStages + s), last_use[x][s] & 1, p.wait_limit_ns, p.status);
       }
     }
   } else if (warp == 1) {
@@ -527,13 +538,29 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         // V operand: the latent c blocks (MLA) or the V blocks (dense), MN-major.
         const uint32_t sv = st0 + (jj % kStages) * kStage + (kMla ? 0u : 2 * C::kBlkRows);
         const uint32_t a_t = tmem + ((jj & 1) ? C::kTmemS1 : C::kTmemS0);
+        if constexpr (C::kParts == 2) {
+          // Two halves of the latent columns; part X of the stage is free after the first.
+          constexpr uint32_t kIdHalf = idesc_bf16_f32(128, 64 * C::kNbX, false, true);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          const uint64_t bd = smem_desc(sv + k * 2048, C::kBlkRows, 1024, kSw128);
-          umma_ts(tmem + kTmemO, a_t + k * 8, bd, kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int k = 0; k < kBN / 16; ++k) {
+              const uint64_t bd = smem_desc(sv + half * C::kNbX * C::kBlkRows + k * 2048, C::kBlkRows, 1024, kSw128);
+              umma_ts(tmem + kTmemO + half * 64 * C::kNbX, a_t + k * 8, bd, kIdHalf, (jj > 0 || k > 0) ? 1u : 0u);
+            }
+            if (half == 0) umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
+          }
+          umma_commit(bar_addr(bars, B_PV));
+          umma_commit(bar_addr(bars, B_KVE0 + kStages + jj % kStages));
+        } else {
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            const uint64_t bd = smem_desc(sv + k * 2048, C::kBlkRows, 1024, kSw128);
+            umma_ts(tmem + kTmemO, a_t + k * 8, bd, kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_addr(bars, B_PV));
+          umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
         }
-        umma_commit(bar_addr(bars, B_PV));
-        umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
         return true;
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
@@ -546,15 +573,24 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         if constexpr (kMla) {
           // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
           // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
-          // share offsets.
+          // share offsets.  With a stage in two parts the K steps run in the order
+          // part X (its content blocks, then the rope block), then part Y.
           constexpr int kCs = 4 * C::kNb;
+          constexpr int kCx = 4 * C::kNbX;  // content steps in part X
 #pragma unroll
-          for (int k = 0; k < kCs + 2; ++k) {
+          for (int n = 0; n < kCs + 2; ++n) {
+            const int k = C::kParts == 2 ? (n < kCx ? n : n < kCx + 2 ? kCs + (n - kCx) : n - 2) : n;
+            if (C::kParts == 2 && n == kCx + 2) {
+              ok = mbar_wait(bar_addr(bars, B_KVF0 + kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
+              if (!ok) break;
+              tc_fence_after();
+            }
             const uint32_t off = k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32;
             const uint32_t sbo = k < kCs ? 1024 : 512;
             const uint32_t lay = k < kCs ? kSw128 : kSw64;
-            umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
+            umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, n > 0);
           }
+          if (!ok) break;
         } else {
           // S = Q . K^T with Q from TMEM: 8 steps over the 128B-swizzled content key
           // blocks (+2 over the 64B-swizzled rope block for the materialised variant).
@@ -575,6 +611,8 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
           constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
           const int sw = n_tiles % kStages;
           ok = mbar_wait(bar_addr(bars, B_KVF0 + sw), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
+               (C::kParts == 1 ||
+                mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma)) &&
                mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
           if (ok) {
             tc_fence_after();
