@@ -73,12 +73,13 @@ struct Cfg<kKindMla, kDcT> {
   static constexpr uint32_t kQaBytes = kStage;                   // Qa tile, same block structure
   static constexpr int kOCols = kDcT;
   static constexpr uint32_t kTmemS0 = 256, kTmemS1 = 384;
-  // With only two stages (d_c = 256) each stage is filled and released in two
-  // parts: X = content blocks [0, d_c/128) + the rope block, Y = the other content
-  // blocks.  P.C then runs as two N = d_c/2 halves, and X is refilled while the
-  // second half runs; the next score tile starts on X and waits for Y last.
-  static constexpr int kParts = kStages == 2 ? 2 : 1;
-  static constexpr int kNbX = kParts == 2 ? kNb / 2 : kNb;  // content blocks in part X
+  // With only two stages (d_c = 256) each stage is filled and released in three
+  // parts with their own barriers: R = the rope block (free once the tile's scores
+  // are done), X = content blocks [0, d_c/128) and Y = the other content blocks.
+  // P.C runs as two N = d_c/2 halves, X is refilled while the second half runs,
+  // and the next score tile takes its K steps in the order R, X, Y.
+  static constexpr int kParts = kStages == 2 ? 3 : 1;
+  static constexpr int kNbX = kParts == 3 ? kNb / 2 : kNb;  // content blocks in part X
 };
 
 // Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
@@ -473,17 +474,22 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         const uint32_t sa = st0 + st * kStage;
         if (use == 0 && kMla && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
         for (int x = 0; ok && x < kParts; ++x) {
+          // Three-part stages: the W_UV item has no rope part (and is the stage's last use).
+          if (kParts == 3 && x == 0 && i == n_tiles) continue;
           if (use > 0) ok = mbar_wait(bar_addr(bars, B_KVE0 + x * kStages + st), (use - 1) & 1, ctl,
                                       kDevTimeoutProducer);
           if (!ok) break;
           const uint32_t fb = bar_addr(bars, B_KVF0 + x * kStages + st);
           const int kv0 = i * kBN;
           if constexpr (kMla) {
-            const int blo = x == 0 ? 0 : C::kNbX, bhi = x == 0 ? C::kNbX : C::kNb;
+            // part x: content blocks [blo, bhi) and (rope) the 64B-swizzled rope block
+            const int blo = kParts == 1 ? 0 : x == 2 ? C::kNbX : 0;
+            const int bhi = kParts == 1 ? C::kNb : x == 0 ? 0 : x == 1 ? C::kNbX : C::kNb;
+            const bool rope = kParts == 1 || x == 0;
             if (i < n_tiles) {
-              mbar_arrive_expect_tx(fb, (bhi - blo) * C::kBlkRows + (x == 0 ? 128u * 64u : 0u));
+              mbar_arrive_expect_tx(fb, (bhi - blo) * C::kBlkRows + (rope ? 128u * 64u : 0u));
               for (int blk = blo; blk < bhi; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
-              if (x == 0) tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
+              if (rope) tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
             } else {
               mbar_arrive_expect_tx(fb, (bhi - blo) * kBlk128);
               for (int blk = blo; blk < bhi; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
@@ -538,8 +544,9 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         // V operand: the latent c blocks (MLA) or the V blocks (dense), MN-major.
         const uint32_t sv = st0 + (jj % kStages) * kStage + (kMla ? 0u : 2 * C::kBlkRows);
         const uint32_t a_t = tmem + ((jj & 1) ? C::kTmemS1 : C::kTmemS0);
-        if constexpr (C::kParts == 2) {
-          // Two halves of the latent columns; part X of the stage is free after the first.
+        if constexpr (C::kParts == 3) {
+          // Two halves of the latent columns; part X of the stage is free after the
+          // first, part Y after the second.
           constexpr uint32_t kIdHalf = idesc_bf16_f32(128, 64 * C::kNbX, false, true);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -548,10 +555,10 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
               const uint64_t bd = smem_desc(sv + half * C::kNbX * C::kBlkRows + k * 2048, C::kBlkRows, 1024, kSw128);
               umma_ts(tmem + kTmemO + half * 64 * C::kNbX, a_t + k * 8, bd, kIdHalf, (jj > 0 || k > 0) ? 1u : 0u);
             }
-            if (half == 0) umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
+            if (half == 0) umma_commit(bar_addr(bars, B_KVE0 + kStages + jj % kStages));
           }
           umma_commit(bar_addr(bars, B_PV));
-          umma_commit(bar_addr(bars, B_KVE0 + kStages + jj % kStages));
+          umma_commit(bar_addr(bars, B_KVE0 + 2 * kStages + jj % kStages));
         } else {
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k) {
@@ -573,15 +580,17 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         if constexpr (kMla) {
           // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
           // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
-          // share offsets.  With a stage in two parts the K steps run in the order
-          // part X (its content blocks, then the rope block), then part Y.
+          // share offsets.  With a stage in three parts the K steps run in the order
+          // R (the rope block), X, Y, each part waited for just before its steps,
+          // and R is released as soon as the scores are done.
           constexpr int kCs = 4 * C::kNb;
           constexpr int kCx = 4 * C::kNbX;  // content steps in part X
 #pragma unroll
           for (int n = 0; n < kCs + 2; ++n) {
-            const int k = C::kParts == 2 ? (n < kCx ? n : n < kCx + 2 ? kCs + (n - kCx) : n - 2) : n;
-            if (C::kParts == 2 && n == kCx + 2) {
-              ok = mbar_wait(bar_addr(bars, B_KVF0 + kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
+            const int k = C::kParts == 3 ? (n < 2 ? kCs + n : n - 2) : n;
+            if (C::kParts == 3 && (n == 2 || n == 2 + kCx)) {  // (part R was waited for above)
+              const int x = n == 2 ? 1 : 2;
+              ok = mbar_wait(bar_addr(bars, B_KVF0 + x * kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
               if (!ok) break;
               tc_fence_after();
             }
@@ -591,6 +600,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, n > 0);
           }
           if (!ok) break;
+          if constexpr (C::kParts == 3) umma_commit(bar_addr(bars, B_KVE0 + st));  // R free once S is done
         } else {
           // S = Q . K^T with Q from TMEM: 8 steps over the 128B-swizzled content key
           // blocks (+2 over the 64B-swizzled rope block for the materialised variant).
@@ -610,9 +620,12 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         if (ok) {
           constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
           const int sw = n_tiles % kStages;
-          ok = mbar_wait(bar_addr(bars, B_KVF0 + sw), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma) &&
-               (C::kParts == 1 ||
-                mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), (n_tiles / kStages) & 1, ctl, kDevTimeoutMma)) &&
+          // W_UV_h blocks: the whole stage, or parts X and Y of a three-part stage.
+          const int ph = (n_tiles / kStages) & 1;
+          ok = (C::kParts == 1
+                    ? mbar_wait(bar_addr(bars, B_KVF0 + sw), ph, ctl, kDevTimeoutMma)
+                    : mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), ph, ctl, kDevTimeoutMma) &&
+                          mbar_wait(bar_addr(bars, B_KVF0 + 2 * kStages + sw), ph, ctl, kDevTimeoutMma)) &&
                mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
           if (ok) {
             tc_fence_after();
