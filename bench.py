@@ -401,6 +401,31 @@ def run_ours(args, w, rank, world, local_rank):
     dense_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in dense_ev), dist, dev) / args.steps
     del kd, vd, out_d
 
+    # ---- the same attention with the last partial wave split over key ranges
+    ws_bytes = vm.vmla_chunk_attention_splitkv_workspace_bytes(w.batch, w.n_q, w.heads, w.n_kv)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    out_s = torch.empty_like(q)
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        vm.vmla_chunk_attention_splitkv(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                        out_s, workspace=ws, stream=stream)
+    sk_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush_buf.zero_()
+        sk_ev[k][0].record(stream)
+        vm.vmla_chunk_attention_splitkv(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE,
+                                        out_s, workspace=ws, stream=stream)
+        sk_ev[k][1].record(stream)
+    barrier()
+    vm.vmla_get_device_status(stream)
+    splitkv_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in sk_ev), dist, dev) / args.steps
+    splitkv = {"ms": splitkv_ms, "tflops": w.attention_flops() / (splitkv_ms * 1e-3) / 1e12,
+               "workspace_bytes": ws_bytes,
+               "note": "vmla_chunk_attention_splitkv: the last partial wave of units split over key ranges "
+                       "(no split when the units fill whole waves)"}
+    del ws, out_s
+
     # ---- non-absorbed form on the same cache and queries: materialise K_h / V_h, then attend
     kvm = torch.empty(w.batch, w.n_kv, 2 * w.heads, w.d_head, dtype=torch.bfloat16, device=dev)
     out_m = torch.empty_like(q)
@@ -597,6 +622,7 @@ def run_ours(args, w, rank, world, local_rank):
         "pct_bf16_nominal_2250": 100.0 * achieved / 2250.0,
         "attention_layer_tokens_per_s": w.batch * w.n_q / (attn_mean * 1e-3),
         "nonabsorbed": nonabsorbed,
+        "splitkv": splitkv,
         "projections": projections,
         "dc_sweep": dc_sweep,
         "dense": {"ms": dense_ms, "tflops": w.dense_flops() / (dense_ms * 1e-3) / 1e12,
@@ -766,10 +792,14 @@ def single_layer_figures(vm, w, dev, dist, reps, warmup, local_rank=0, seed=0):
     kvm = torch.empty(w.batch, w.n_kv, 2 * H, w.d_head, dtype=torch.bfloat16, device=dev)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    ws_bytes = vm.vmla_chunk_attention_splitkv_workspace_bytes(w.batch, w.n_q, H, w.n_kv)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     calls = {
         "append": lambda: vm.vmla_cache_append(x_chunk, wd, wk, cache, w.n_cached, w.chunk_t0, w.grid_h, w.grid_w),
         "attention": lambda: vm.vmla_chunk_attention(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h,
                                                      w.grid_w, SCALE, out),
+        "attention_splitkv": lambda: vm.vmla_chunk_attention_splitkv(q, qr, wuk, wuv, cache, w.n_kv, w.chunk_t0,
+                                                                     w.grid_h, w.grid_w, SCALE, out, workspace=ws),
         "materialize": lambda: vm.vmla_materialize_kv(wuk, wuv, cache, w.n_kv, kvm),
         "attention_materialized": lambda: vm.vmla_chunk_attention_materialized(
             q, qr, kvm, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE, out),
@@ -806,6 +836,11 @@ def single_layer_figures(vm, w, dev, dist, reps, warmup, local_rank=0, seed=0):
                      f"H={H}x{w.d_head}, d_c={w.d_c}, d_r={w.d_r}"),
         "reps": reps,
         "attention": {"ms": ms["attention"], "tflops": w.attention_flops() / (ms["attention"] * 1e-3) / 1e12},
+        "attention_splitkv": {"ms": ms["attention_splitkv"],
+                              "tflops": w.attention_flops() / (ms["attention_splitkv"] * 1e-3) / 1e12,
+                              "workspace_bytes": ws_bytes,
+                              "note": "the last partial wave of (sample, query tile, head) units split over key "
+                                      "ranges (no split when the units fill whole waves)"},
         "append": {"us": ms["append"] * 1e3},
         "nonabsorbed": {"ms_materialize": ms["materialize"], "ms_attention": ms["attention_materialized"],
                         "ms_total": ms["materialize"] + ms["attention_materialized"],
@@ -814,7 +849,7 @@ def single_layer_figures(vm, w, dev, dist, reps, warmup, local_rank=0, seed=0):
         "clocks_attention": clocks,
         "inputs": "drawn on the device (torch normal, seeded); timing only",
     }
-    del cache, q, qr, out, kd, vd, kvm, flush_w, flush_r
+    del cache, q, qr, out, kd, vd, kvm, flush_w, flush_r, ws
     torch.cuda.empty_cache()
     return res
 

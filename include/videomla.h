@@ -101,13 +101,49 @@ vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const ui
  * (bidirectional inside the chunk).  W_UK is absorbed into the queries and
  * W_UV is applied once per query after the latent accumulation; bf16 tensor-core
  * products with fp32 accumulation.
- * Limits: 1 <= n_kv <= cap < 2^31; n_q >= 1; heads >= 1; scale > 0 and finite.
+ * Limits: 1 <= n_kv <= cap < 2^31; n_q >= 1; heads >= 1; scale > 0 and finite;
+ * batch * ceil(n_q / 128) * heads * 8 < 2^31.
  */
 vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
                                  const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
                                  int32_t n_q, int32_t heads, int64_t cap, int64_t n_kv,
                                  int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
                                  uint16_t* out, void* stream);
+
+/*
+ * vmla_chunk_attention_splitkv -- vmla_chunk_attention with a caller workspace that
+ * lets the launch split work along the keys.  (Same computation as above; the split
+ * is a scheduling choice of this library, with no counterpart on the pages.)
+ *
+ * The launch has one unit of work per (sample, 128-query tile, head), and one unit
+ * runs on one SM at a time.  When the units do not fill the last wave of SMs, each
+ * unit of that partial wave runs as `split` parts (2 <= split <= 8, each over at
+ * least 32 key tiles of 128 keys, so windows under 8192 keys never split) over
+ * consecutive key ranges: every part writes its
+ * unnormalised latent accumulation with its running maximum and sum to the workspace,
+ * and the part that finishes last rescales all parts to a common maximum, sums them
+ * and applies W_UV.  split is chosen to minimise ceil(split * rest / SMs) / split,
+ * the tail's length in units of one whole unit.  Results equal vmla_chunk_attention's
+ * up to fp32 summation order.
+ *
+ * vmla_chunk_attention_splitkv_workspace_bytes -- bytes of workspace the call needs on
+ * the current device for these sizes: 0 when the units fill whole waves (or a split
+ * would not shorten the tail), so that the call needs no workspace; -1 on bad sizes
+ * or when no device is current.
+ *
+ * workspace: caller-owned device memory of at least that many bytes, 16-byte aligned
+ * (may be NULL when 0 bytes are needed).  Its contents on entry do not matter: the
+ * call clears the arrival counters it holds with an asynchronous memset on `stream`
+ * before the launch.  Calls sharing one workspace must not overlap on the GPU.
+ * Errors: VMLA_ERR_INVALID_ARG when the workspace is missing or smaller than needed.
+ */
+int64_t vmla_chunk_attention_splitkv_workspace_bytes(int32_t batch, int32_t n_q, int32_t heads, int64_t n_kv);
+
+vmla_status vmla_chunk_attention_splitkv(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                         const uint16_t* w_uv, const uint16_t* cache, int32_t batch, int32_t n_q,
+                                         int32_t heads, int64_t cap, int64_t n_kv, int64_t t0, int32_t grid_h,
+                                         int32_t grid_w, float scale, void* workspace, int64_t workspace_bytes,
+                                         uint16_t* out, void* stream);
 
 /*
  * The same two calls for another latent width d_c (summary "Key results": batch

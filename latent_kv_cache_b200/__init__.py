@@ -72,6 +72,11 @@ def _load():
     lib.vmla_chunk_attention_nonabsorbed_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32,
                                                              f32, P, P]
     lib.vmla_chunk_attention_nonabsorbed_noalloc.restype = ctypes.c_int
+    lib.vmla_chunk_attention_splitkv_workspace_bytes.argtypes = [i32, i32, i32, i64]
+    lib.vmla_chunk_attention_splitkv_workspace_bytes.restype = i64
+    lib.vmla_chunk_attention_splitkv.argtypes = [P, P, P, P, P, i32, i32, i32, i64, i64, i64, i32, i32, f32, P, i64,
+                                                 P, P]
+    lib.vmla_chunk_attention_splitkv.restype = ctypes.c_int
     return lib
 
 
@@ -248,6 +253,39 @@ def vmla_chunk_attention_nonabsorbed(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0
                                                 int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
                                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                                 _ptr(out, "out"), _stream(stream)))
+
+
+def vmla_chunk_attention_splitkv_workspace_bytes(batch: int, n_q: int, heads: int, n_kv: int) -> int:
+    """Workspace bytes vmla_chunk_attention_splitkv needs on the current device (0: none)."""
+    n = lib.vmla_chunk_attention_splitkv_workspace_bytes(int(batch), int(n_q), int(heads), int(n_kv))
+    if n < 0:
+        raise ValueError("bad sizes or no current CUDA device")
+    return n
+
+
+def vmla_chunk_attention_splitkv(q, q_rope, w_uk, w_uv, cache, n_kv: int, t0: int, grid_h: int, grid_w: int,
+                                 scale: float, out, workspace=None, stream=None) -> None:
+    """vmla_chunk_attention whose last partial wave of (sample, query tile, head) units may
+    run split over key ranges.  workspace: a contiguous CUDA tensor of at least
+    vmla_chunk_attention_splitkv_workspace_bytes(B, Nq, H, n_kv) bytes; when None, one of
+    that size is taken from torch's allocator for this call."""
+    B, Nq, H, dh = q.shape
+    if dh != D_HEAD or tuple(q_rope.shape) != (B, Nq, H, D_R) or tuple(out.shape) != (B, Nq, H, D_HEAD):
+        raise ValueError("q/q_rope/out shapes do not match [B, Nq, H, 128|32]")
+    if tuple(w_uk.shape) != (H * D_HEAD, D_C) or tuple(w_uv.shape) != (H * D_HEAD, D_C):
+        raise ValueError("w_uk / w_uv must be [H*128, 192]")
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D_C + D_R:
+        raise ValueError("cache must be [B, cap, 224]")
+    if workspace is None:
+        need = vmla_chunk_attention_splitkv_workspace_bytes(B, Nq, H, n_kv)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check(lib.vmla_chunk_attention_splitkv(_ptr(q, "q"), _ptr(q_rope, "q_rope"), _ptr(w_uk, "w_uk"),
+                                            _ptr(w_uv, "w_uv"), _ptr(cache, "cache"), B, Nq, H, cache.shape[1],
+                                            int(n_kv), int(t0), int(grid_h), int(grid_w), float(scale),
+                                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                            _ptr(out, "out"), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

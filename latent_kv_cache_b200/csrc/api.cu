@@ -16,7 +16,8 @@ cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, co
                                    const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
                                    int heads, int d_c, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
                                    int grid_w, float scale, uint16_t* out, int* status,
-                                   cudaStream_t stream, bool* encode_failed);
+                                   cudaStream_t stream, bool* encode_failed, const SplitPlan& plan,
+                                   void* workspace);
 cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int batch,
                                    int n_q, int64_t n_kv, int heads, float scale, uint16_t* out,
                                    int* status, cudaStream_t stream, bool* encode_failed);
@@ -116,35 +117,72 @@ vmla_status vmla_cache_append(const uint16_t* x, const uint16_t* w_dkv, const ui
                               grid_w, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Units of the latent attention launch: (sample, query tile, head).
+int64_t latent_units(int32_t batch, int32_t n_q, int32_t heads) {
+  return (int64_t)batch * ((n_q + 127) / 128) * heads;
+}
+
+// Shared body of the latent-attention entry points.  split: may run the last
+// partial wave's units as key-range parts merged through `workspace`.
+vmla_status chunk_attention_impl(const char* who, const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                 const uint16_t* w_uv, const uint16_t* cache, int32_t batch, int32_t n_q,
+                                 int32_t heads, int32_t d_c, int64_t cap, int64_t n_kv, int64_t t0, int32_t grid_h,
+                                 int32_t grid_w, float scale, bool split, void* workspace, int64_t workspace_bytes,
+                                 uint16_t* out, void* stream) {
+  if (!supported_dc(d_c)) return fail(VMLA_ERR_UNSUPPORTED, "%s: d_c must be 64, 128, 192 or 256", who);
+  if (!aligned16(q) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(w_uv) ||
+      !aligned16(cache) || !aligned16(out))
+    return fail(VMLA_ERR_INVALID_ARG, "%s: pointers must be non-null and 16-byte aligned", who);
+  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "%s: batch must be in [1, 65535]", who);
+  if (n_q < 1) return fail(VMLA_ERR_INVALID_ARG, "%s: n_q must be >= 1", who);
+  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "%s: heads must be in [1, 512]", who);
+  if (n_kv < 1 || n_kv > cap) return fail(VMLA_ERR_INVALID_ARG, "%s: need 1 <= n_kv <= cap", who);
+  if (cap >= (int64_t(1) << 31)) return fail(VMLA_ERR_UNSUPPORTED, "%s: cap must be < 2^31", who);
+  if (latent_units(batch, n_q, heads) * vmla::kMaxSplit > 0x7FFFFFFF)
+    return fail(VMLA_ERR_UNSUPPORTED, "%s: too many query tiles x heads x samples", who);
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(VMLA_ERR_INVALID_ARG, "%s: scale must be positive and finite", who);
+  vmla_status st = check_positions(n_q, t0, grid_h, grid_w);
+  if (st != VMLA_OK) return st;
+  int* status = vmla::device_status_word();
+  if (!status) return fail(VMLA_ERR_CUDA, "%s: no CUDA device", who);
+  const int64_t units = latent_units(batch, n_q, heads);
+  vmla::SplitPlan plan{units, 1, 0};
+  if (split) {
+    plan = vmla::plan_split(units, (int)((n_kv + 127) / 128), vmla::sm_count_current_device());
+    const int64_t need = vmla::split_workspace_bytes(plan, d_c);
+    if (need > 0) {
+      if (!aligned16(workspace))
+        return fail(VMLA_ERR_INVALID_ARG, "%s: workspace must be non-null and 16-byte aligned", who);
+      if (workspace_bytes < need)
+        return fail(VMLA_ERR_INVALID_ARG, "%s: workspace of %lld bytes, need %lld", who, (long long)workspace_bytes,
+                    (long long)need);
+    }
+  }
+  bool enc_fail = false;
+  cudaError_t e = vmla::launch_chunk_attention(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, d_c, cap,
+                                               n_kv, t0, grid_h, grid_w, scale, out, status,
+                                               static_cast<cudaStream_t>(stream), &enc_fail, plan, workspace);
+  if (enc_fail) return fail(VMLA_ERR_CUDA, "%s: tensor-map encoding failed", who);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
+  return VMLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 vmla_status vmla_chunk_attention_dc(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
                                     const uint16_t* w_uv, const uint16_t* cache, int32_t batch,
                                     int32_t n_q, int32_t heads, int32_t d_c, int64_t cap, int64_t n_kv,
                                     int64_t t0, int32_t grid_h, int32_t grid_w, float scale,
                                     uint16_t* out, void* stream) {
-  if (!supported_dc(d_c)) return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: d_c must be 64, 128, 192 or 256");
-  if (!aligned16(q) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(w_uv) ||
-      !aligned16(cache) || !aligned16(out))
-    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: pointers must be non-null and 16-byte aligned");
-  if (batch < 1 || batch > 65535) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: batch must be in [1, 65535]");
-  if (n_q < 1) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: n_q must be >= 1");
-  if (heads < 1 || heads > 512) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: heads must be in [1, 512]");
-  if (n_kv < 1 || n_kv > cap) return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: need 1 <= n_kv <= cap");
-  if (cap >= (int64_t(1) << 31)) return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: cap must be < 2^31");
-  if ((int64_t)((n_q + 127) / 128) * heads > 0x7FFFFFFF)
-    return fail(VMLA_ERR_UNSUPPORTED, "chunk_attention: too many query tiles");
-  if (!(scale > 0.0f) || !std::isfinite(scale))
-    return fail(VMLA_ERR_INVALID_ARG, "chunk_attention: scale must be positive and finite");
-  vmla_status st = check_positions(n_q, t0, grid_h, grid_w);
-  if (st != VMLA_OK) return st;
-  int* status = vmla::device_status_word();
-  if (!status) return fail(VMLA_ERR_CUDA, "chunk_attention: no CUDA device");
-  bool enc_fail = false;
-  cudaError_t e = vmla::launch_chunk_attention(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, d_c, cap,
-                                               n_kv, t0, grid_h, grid_w, scale, out, status,
-                                               static_cast<cudaStream_t>(stream), &enc_fail);
-  if (enc_fail) return fail(VMLA_ERR_CUDA, "chunk_attention: tensor-map encoding failed");
-  if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
-  return VMLA_OK;
+  return chunk_attention_impl("chunk_attention", q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, d_c, cap, n_kv,
+                              t0, grid_h, grid_w, scale, false, nullptr, 0, out, stream);
 }
 
 vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
@@ -154,6 +192,26 @@ vmla_status vmla_chunk_attention(const uint16_t* q, const uint16_t* q_rope, cons
                                  uint16_t* out, void* stream) {
   return vmla_chunk_attention_dc(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, vmla::kDc, cap, n_kv, t0,
                                  grid_h, grid_w, scale, out, stream);
+}
+
+int64_t vmla_chunk_attention_splitkv_workspace_bytes(int32_t batch, int32_t n_q, int32_t heads, int64_t n_kv) {
+  if (batch < 1 || batch > 65535 || n_q < 1 || heads < 1 || heads > 512 || n_kv < 1 || n_kv >= (int64_t(1) << 31))
+    return -1;
+  if (latent_units(batch, n_q, heads) * vmla::kMaxSplit > 0x7FFFFFFF) return -1;
+  const int sms = vmla::sm_count_current_device();
+  if (sms <= 0) return -1;
+  const vmla::SplitPlan plan =
+      vmla::plan_split(latent_units(batch, n_q, heads), (int)((n_kv + 127) / 128), sms);
+  return vmla::split_workspace_bytes(plan, vmla::kDc);
+}
+
+vmla_status vmla_chunk_attention_splitkv(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
+                                         const uint16_t* w_uv, const uint16_t* cache, int32_t batch, int32_t n_q,
+                                         int32_t heads, int64_t cap, int64_t n_kv, int64_t t0, int32_t grid_h,
+                                         int32_t grid_w, float scale, void* workspace, int64_t workspace_bytes,
+                                         uint16_t* out, void* stream) {
+  return chunk_attention_impl("chunk_attention_splitkv", q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, vmla::kDc,
+                              cap, n_kv, t0, grid_h, grid_w, scale, true, workspace, workspace_bytes, out, stream);
 }
 
 vmla_status vmla_dense_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,

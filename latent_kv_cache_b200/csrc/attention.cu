@@ -141,10 +141,11 @@ enum Bar {
   B_SF0 = B_KVE0 + 8, B_SF1,
   B_PF0, B_PF1,
   B_PV, B_OA, B_OUT, B_DRAIN,
+  B_PART, B_LAST,           // split key range: partial written / last-part decision made
   B_MX0,                    // 8 barriers: (TMEM lane quadrant, tile parity)
   B_COUNT = B_MX0 + 8
 };
-static_assert(B_COUNT * 8 + 8 <= 512, "barrier area");
+static_assert(B_COUNT * 8 + 16 <= 512, "barrier area");
 
 struct ChunkMaps {
   CUtensorMap q;    // [B, Nq, H, 128] box (64, 1, 128, 1), 128B swizzle
@@ -178,6 +179,17 @@ struct AttnParams {
   int grid_h;
   int grid_w;
   float scale_log2;
+  // Latent kernel work split (1-D grid over units = (sample, query tile, head),
+  // heads fastest).  Units [0, n_full) run whole, one CTA each.  Every later unit
+  // runs as `split` CTAs over consecutive key-tile ranges; each writes its
+  // unnormalised O_lat and its (running max, sum) to the workspace and counts
+  // itself in; the part that arrives last merges all parts and runs the W_UV
+  // epilogue.
+  int n_full;
+  int split;
+  float* ws_o;    // [tail units * split][128][d_c] fp32
+  float* ws_ml;   // [tail units * split][128][2] fp32: running max (log2 units), sum
+  int* ws_cnt;    // [tail units] arrival counters, zero when the launch starts
 };
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, int i) { return base + 8u * i; }
@@ -243,8 +255,10 @@ __device__ __forceinline__ bool exchange(const SoftmaxThread& t, uint32_t bars, 
 }
 
 // Softmax step for key tile j.  Returns false on abort.
+// j: tile index within this CTA's key range (barrier phases); jabs: the tile's
+// index in the key sequence (masking of keys >= n_kv).
 template <int kKind, int kDcT>
-__device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const SoftmaxThread& t,
+__device__ __forceinline__ bool softmax_tile(int j, int jabs, uint32_t bars, const SoftmaxThread& t,
                                              const AttnParams& p, const WaitCtl& ctl,
                                              float& m_run, float& l_part) {
   using C = Cfg<kKind, kDcT>;
@@ -265,7 +279,7 @@ __device__ __forceinline__ bool softmax_tile(int j, uint32_t bars, const Softmax
 #pragma unroll
     for (int e = 0; e < kW - 32; ++e) s[32 + e] = __uint_as_float(rb[e]);
   }
-  const int64_t kv0 = (int64_t)j * C::kBN + kW * t.half;
+  const int64_t kv0 = (int64_t)jabs * C::kBN + kW * t.half;
   if (kv0 + kW > p.n_kv) {
     const int64_t valid = p.n_kv - kv0;  // may be <= 0: the whole half is padding
 #pragma unroll
@@ -395,6 +409,8 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
   const uint32_t bars = qa + L::kBarOff;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);  // split: this part merges
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(tmem_holder + 3);  // split: no W_UV epilogue
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);
 
   const int warp = threadIdx.x >> 5;
@@ -404,10 +420,29 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
   // kernels: query tiles fastest, so the CTAs that run together share one head's
   // key/value tiles and each head's keys and values cross HBM about once.
   const int n_qt = (p.n_q + kBM - 1) / kBM;
-  const int h = kMla ? (int)(blockIdx.x % p.heads) : (int)(blockIdx.x / n_qt);
-  const int q0 = (kMla ? (int)(blockIdx.x / p.heads) : (int)(blockIdx.x % n_qt)) * kBM;
-  const int b = blockIdx.y;
-  const int n_tiles = p.n_kv_tiles;
+  int h, q0, b, unit = 0, part = 0, split = 1;
+  if constexpr (kMla) {
+    // 1-D grid: whole units first, then the parts of the split units.
+    const int u = (int)blockIdx.x;
+    if (u < p.n_full) {
+      unit = u;
+    } else {
+      unit = p.n_full + (u - p.n_full) / p.split;
+      part = (u - p.n_full) % p.split;
+      split = p.split;
+    }
+    const int per_b = n_qt * p.heads;
+    b = unit / per_b;
+    h = (unit % per_b) % p.heads;
+    q0 = ((unit % per_b) / p.heads) * kBM;
+  } else {
+    h = (int)(blockIdx.x / n_qt);
+    q0 = (int)(blockIdx.x % n_qt) * kBM;
+    b = (int)blockIdx.y;
+  }
+  // This CTA's key tiles: [kt0, kt0 + n_tiles) of the n_kv_tiles tiles.
+  const int kt0 = (int)((int64_t)part * p.n_kv_tiles / split);
+  const int n_tiles = (int)((int64_t)(part + 1) * p.n_kv_tiles / split) - kt0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_addr(bars, B_PRO), 1);
@@ -425,8 +460,12 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     mbar_init(bar_addr(bars, B_OA), kSoftmaxThreads);
     mbar_init(bar_addr(bars, B_OUT), 1);
     mbar_init(bar_addr(bars, B_DRAIN), 1);
+    mbar_init(bar_addr(bars, B_PART), kSoftmaxThreads);
+    mbar_init(bar_addr(bars, B_LAST), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar_addr(bars, B_MX0 + i), 64);
     *abort_flag = 0;
+    *last_flag = 0;
+    *skip_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -480,7 +519,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
                                       kDevTimeoutProducer);
           if (!ok) break;
           const uint32_t fb = bar_addr(bars, B_KVF0 + x * kStages + st);
-          const int kv0 = i * kBN;
+          const int kv0 = (kt0 + i) * kBN;
           if constexpr (kMla) {
             // part x: content blocks [blo, bhi) and (rope) the 64B-swizzled rope block
             const int blo = kParts == 1 ? 0 : x == 2 ? C::kNbX : 0;
@@ -627,7 +666,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
                     : mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), ph, ctl, kDevTimeoutMma) &&
                           mbar_wait(bar_addr(bars, B_KVF0 + 2 * kStages + sw), ph, ctl, kDevTimeoutMma)) &&
                mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
-          if (ok) {
+          if (ok && !*skip_flag) {  // (a part of a split unit that does not merge skips it)
             tc_fence_after();
             const uint32_t wb = st0 + sw * kStage;
             // out = O_lat/l . W_UV_h^T (M 128, N 128, K d_c): A from TMEM, W_UV K-major.
@@ -718,7 +757,8 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       mbar_arrive(bar_addr(bars, B_QA));
     }
     float m_run = -INFINITY, l_part = 0.0f;
-    for (int j = 0; ok && j < n_tiles; ++j) ok = softmax_tile<kKind, kDcT>(j, bars, t, p, ctl, m_run, l_part);
+    for (int j = 0; ok && j < n_tiles; ++j)
+      ok = softmax_tile<kKind, kDcT>(j, kt0 + j, bars, t, p, ctl, m_run, l_part);
     float l_other = 0.0f;
     if (ok) ok = exchange(t, bars, n_tiles, l_part, l_other, ctl);
     if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
@@ -728,22 +768,96 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
       uint32_t v[32];
       if constexpr (kMla) {
-        // Normalised O_lat -> bf16 A operand of the W_UV MMA (this half: latent
-        // [d_c/2 half, +d_c/2), i.e. d_c/4 cells).
+        // Split unit: write this part's partial, count it in, and find out whether
+        // this part is the last of its unit (it then merges all parts).
+        bool merge = false, emit = true;
+        int slot0 = 0;
+        if (split > 1) {
+          slot0 = (unit - p.n_full) * split;
+          float* wo = p.ws_o + ((int64_t)(slot0 + part) * kBM + t.r) * kDcT + (kDcT / 2) * t.half;
 #pragma unroll
-        for (int c = 0; c < C::kNb; ++c) {
-          tmem_ld32(t.t_row + kTmemO + (kDcT / 2) * t.half + 32 * c, v);
-          tmem_ld_wait();
-          uint32_t pk[16];
+          for (int c = 0; c < C::kNb; ++c) {  // this half's d_c/2 columns, 32 at a time
+            tmem_ld32(t.t_row + kTmemO + (kDcT / 2) * t.half + 32 * c, v);
+            tmem_ld_wait();
+            float4* dst = reinterpret_cast<float4*>(wo + 32 * c);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack2(v[2 * e], v[2 * e + 1], inv_l);
-          tmem_st16(t.t_row + C::kTmemS0 + (kDcT / 4) * t.half + 16 * c, pk);
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+          }
+          if (t.half == 0) {
+            float2* ml = reinterpret_cast<float2*>(p.ws_ml) + (int64_t)(slot0 + part) * kBM + t.r;
+            *ml = make_float2(m_run, l_part + l_other);
+          }
+          __threadfence();
+          mbar_arrive(bar_addr(bars, B_PART));
+          if (t.half == 0 && t.r == 0) {  // one thread counts the CTA in
+            if (mbar_wait(bar_addr(bars, B_PART), 0, ctl, kDevTimeoutSoftmax)) {
+              const int prev = atomicAdd(p.ws_cnt + (unit - p.n_full), 1);
+              *last_flag = prev == split - 1 ? 1 : 0;
+              mbar_arrive(bar_addr(bars, B_LAST));
+            }
+          }
+          ok = warp_wait(bar_addr(bars, B_LAST), 0, ctl);
+          merge = ok && *last_flag != 0;
+          emit = merge;
+          if (merge) __threadfence();
+          if (!emit) *skip_flag = 1;
         }
-        tmem_st_wait();
+        if (ok && emit) {
+          // Normalised O_lat -> bf16 A operand of the W_UV MMA (this half: latent
+          // [d_c/2 half, +d_c/2), i.e. d_c/4 cells).  Merging: the parts' O_lat
+          // are brought to the common reference max and summed, over the summed l.
+          const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + (int64_t)slot0 * kBM + t.r;
+          float w_own = 1.0f, m_tot = m_run, scale_l = inv_l;
+          if (merge) {
+            for (int r2 = 0; r2 < split; ++r2)
+              if (r2 != part) m_tot = fmaxf(m_tot, __ldcg(&ml[(int64_t)r2 * kBM].x));
+            w_own = exp2f(m_run - m_tot);
+            float l_tot = (l_part + l_other) * w_own;
+            for (int r2 = 0; r2 < split; ++r2) {
+              if (r2 == part) continue;
+              const float2 mlr = __ldcg(&ml[(int64_t)r2 * kBM]);
+              l_tot += mlr.y * exp2f(mlr.x - m_tot);
+            }
+            scale_l = 1.0f / l_tot;
+          }
+#pragma unroll
+          for (int c = 0; c < C::kNb; ++c) {
+            tmem_ld32(t.t_row + kTmemO + (kDcT / 2) * t.half + 32 * c, v);
+            tmem_ld_wait();
+            if (merge) {
+              float acc[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(v[e]) * w_own;
+              for (int r2 = 0; r2 < split; ++r2) {
+                if (r2 == part) continue;
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.ws_o + ((int64_t)(slot0 + r2) * kBM + t.r) * kDcT + (kDcT / 2) * t.half + 32 * c);
+                const float w2 = exp2f(__ldcg(&ml[(int64_t)r2 * kBM].x) - m_tot);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                  const float4 f = __ldcg(src + q4);
+                  acc[4 * q4] = fmaf(f.x, w2, acc[4 * q4]);
+                  acc[4 * q4 + 1] = fmaf(f.y, w2, acc[4 * q4 + 1]);
+                  acc[4 * q4 + 2] = fmaf(f.z, w2, acc[4 * q4 + 2]);
+                  acc[4 * q4 + 3] = fmaf(f.w, w2, acc[4 * q4 + 3]);
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(acc[e]);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack2(v[2 * e], v[2 * e + 1], scale_l);
+            tmem_st16(t.t_row + C::kTmemS0 + (kDcT / 4) * t.half + 16 * c, pk);
+          }
+          tmem_st_wait();
+        }
         tc_fence_before();
-        mbar_arrive(bar_addr(bars, B_OA));
-        ok = warp_wait(bar_addr(bars, B_OUT), 0, ctl);
-        if (ok) {
+        mbar_arrive(bar_addr(bars, B_OA));  // (a part that does not merge only releases the MMA thread)
+        if (ok && emit) ok = warp_wait(bar_addr(bars, B_OUT), 0, ctl);
+        if (ok && emit) {
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -855,11 +969,26 @@ bool make_head_map(CUtensorMap* m, const uint16_t* t, int batch, int64_t n_rows,
 
 namespace {
 
+// Workspace of the split key ranges, laid out [O partials | (m, l) | counters].
+struct SplitLayout {
+  int64_t o_bytes, ml_bytes, cnt_bytes, total;
+};
+SplitLayout split_layout(int64_t tail_units, int split, int d_c) {
+  auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+  SplitLayout l;
+  l.o_bytes = up(tail_units * split * kBM * d_c * 4);
+  l.ml_bytes = up(tail_units * split * kBM * 8);
+  l.cnt_bytes = up(tail_units * 4);
+  l.total = l.o_bytes + l.ml_bytes + l.cnt_bytes;
+  return l;
+}
+
 template <int kDcT>
 cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
                                      const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q, int heads,
                                      int64_t cap, int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale,
-                                     uint16_t* out, int* status, cudaStream_t stream, bool* encode_failed) {
+                                     uint16_t* out, int* status, cudaStream_t stream, bool* encode_failed,
+                                     const SplitPlan& plan, void* workspace) {
   using C = Cfg<kKindMla, kDcT>;
   using L = Layout<kKindMla, kDcT>;
   constexpr int kRow = kDcT + kDr;
@@ -900,36 +1029,95 @@ cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, 
   p.grid_h = grid_h;
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.n_full = (int)plan.n_full;
+  p.split = plan.split;
+  int64_t blocks = plan.n_full;
+  if (plan.split > 1) {
+    const SplitLayout sl = split_layout(plan.tail_units, plan.split, kDcT);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(ws);
+    p.ws_ml = reinterpret_cast<float*>(ws + sl.o_bytes);
+    p.ws_cnt = reinterpret_cast<int*>(ws + sl.o_bytes + sl.ml_bytes);
+    cudaError_t e = cudaMemsetAsync(p.ws_cnt, 0, plan.tail_units * sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+    blocks += plan.tail_units * plan.split;
+  }
   static thread_local RopeTable tab;
   static thread_local RopeTableKey tab_key;
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
-  dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_chunk_attn<kDcT><<<grid, kThreads, L::kBytes, stream>>>(maps, p, tab);
+  k_chunk_attn<kDcT><<<dim3((unsigned)blocks), kThreads, L::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// d_c in {64, 128, 192, 256}; the caller has validated it.
+int sm_count_current_device() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
+// One latent-attention CTA per SM at a time (shared memory and TMEM).  Units
+// (sample, query tile, head) fill whole waves of `sms`; when the last wave is
+// partial, its units may run as `split` parts over key ranges so that the tail
+// takes ceil(split * rem / sms) / split of a whole unit's time instead of one.
+// Every part repeats the unit's prologue (query tile, q.W_UK) and adds its
+// partial's write, the count-in and the last part's merge, so a part keeps at
+// least kMinPartTiles key tiles: measured on the small workload (5 key tiles,
+// 24 units) a 5-way split took 2.5x the unsplit launch, while at 1080P (574 key
+// tiles, 84 tail units, 7-way) it saved 1.5% in an interleaved A/B.
+SplitPlan plan_split(int64_t units, int n_kv_tiles, int sms) {
+  SplitPlan s{units, 1, 0};
+  if (sms <= 0 || units <= 0) return s;
+  const int64_t full = units / sms * sms, rem = units - full;
+  if (rem == 0) return s;
+  double best = 1.0;
+  for (int k = 2; k <= kMaxSplit && k * kMinPartTiles <= n_kv_tiles; ++k) {
+    const double tail = (double)((k * rem + sms - 1) / sms) / k;
+    if (tail < best - 1e-9) {
+      best = tail;
+      s.split = k;
+    }
+  }
+  if (s.split > 1) {
+    s.n_full = full;
+    s.tail_units = rem;
+  }
+  return s;
+}
+
+int64_t split_workspace_bytes(const SplitPlan& plan, int d_c) {
+  return plan.split > 1 ? split_layout(plan.tail_units, plan.split, d_c).total : 0;
+}
+
+// d_c in {64, 128, 192, 256}; the caller has validated it.  `plan` says which
+// units run whole; with plan.split > 1, `workspace` holds split_workspace_bytes.
 cudaError_t launch_chunk_attention(const uint16_t* q, const uint16_t* q_rope, const uint16_t* w_uk,
                                    const uint16_t* w_uv, const uint16_t* cache, int batch, int n_q,
                                    int heads, int d_c, int64_t cap, int64_t n_kv, int64_t t0, int grid_h,
                                    int grid_w, float scale, uint16_t* out, int* status,
-                                   cudaStream_t stream, bool* encode_failed) {
+                                   cudaStream_t stream, bool* encode_failed, const SplitPlan& plan,
+                                   void* workspace) {
   switch (d_c) {
     case 64:
       return launch_chunk_attention_t<64>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
-                                          grid_w, scale, out, status, stream, encode_failed);
+                                          grid_w, scale, out, status, stream, encode_failed, plan, workspace);
     case 128:
       return launch_chunk_attention_t<128>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
-                                           grid_w, scale, out, status, stream, encode_failed);
+                                           grid_w, scale, out, status, stream, encode_failed, plan, workspace);
     case 192:
       return launch_chunk_attention_t<192>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
-                                           grid_w, scale, out, status, stream, encode_failed);
+                                           grid_w, scale, out, status, stream, encode_failed, plan, workspace);
     case 256:
       return launch_chunk_attention_t<256>(q, q_rope, w_uk, w_uv, cache, batch, n_q, heads, cap, n_kv, t0, grid_h,
-                                           grid_w, scale, out, status, stream, encode_failed);
+                                           grid_w, scale, out, status, stream, encode_failed, plan, workspace);
     default:
       return cudaErrorInvalidValue;
   }

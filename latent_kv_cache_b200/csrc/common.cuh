@@ -38,6 +38,21 @@ struct RopeTableKey {
 // steps share t0 and the grid, and a rollout keeps its grid).
 void build_rope_table(RopeTable* tab, RopeTableKey* key, int64_t t0, int n_frames, int grid_h, int grid_w);
 
+// Work split of the latent attention launch: units (sample, query tile, head)
+// [0, n_full) run whole, one CTA each; the tail_units after them run as `split`
+// CTAs each over consecutive key ranges, merged by the part that finishes last
+// (split == 1: no split).
+struct SplitPlan {
+  int64_t n_full;
+  int split;
+  int64_t tail_units;
+};
+constexpr int kMaxSplit = 8;
+constexpr int kMinPartTiles = 32;  // key tiles of 128 keys per part, at least
+SplitPlan plan_split(int64_t units, int n_kv_tiles, int sms);
+int64_t split_workspace_bytes(const SplitPlan& plan, int d_c);
+int sm_count_current_device();  // 0 when no device is current
+
 // Device-side status word of the current device (lazily looked up, cached per device).
 int* device_status_word();
 

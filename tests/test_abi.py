@@ -128,3 +128,17 @@ def test_materialized_kv_bytes_overflow_is_rejected(vm):
     assert L.vmla_chunk_attention_nonabsorbed_noalloc(A, A, A, A, A, 65535, 192, 512, big, big, 0, 8, 8, f(0.1),
                                                       A, None) == 2
     assert "overflow" in vm.vmla_last_error()
+
+
+def test_splitkv_validation(vm):
+    L = vm.lib
+    f = ctypes.c_float
+    assert L.vmla_chunk_attention_splitkv_workspace_bytes(0, 192, 12, 576) == -1
+    assert L.vmla_chunk_attention_splitkv_workspace_bytes(1, 192, 600, 576) == -1
+    assert L.vmla_chunk_attention_splitkv_workspace_bytes(1, 192, 12, 0) == -1
+    assert L.vmla_chunk_attention_splitkv(A, A, A, A, None, 1, 192, 12, 576, 576, 6, 8, 8, f(0.1), A, 1 << 20, A,
+                                          None) == 1
+    assert L.vmla_chunk_attention_splitkv(A, A, A, A, A, 1, 192, 12, 576, 577, 6, 8, 8, f(0.1), A, 1 << 20, A,
+                                          None) == 1
+    assert L.vmla_chunk_attention_splitkv(A, A, A, A, A, 1, 192, 12, 576, 576, 6, 8, 8, f(0.0), A, 1 << 20, A,
+                                          None) == 1

@@ -158,3 +158,24 @@ def test_canary_append_two_slice_ctas(vm, d_c, n_tok):
     vm.vmla_cache_append_dc(x, to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache, 0, 3, w.grid_h, w.grid_w)
     vm.vmla_get_device_status()
     assert_guards(cbuf, f"append two slice CTAs per SM d_c={d_c}")
+
+
+def test_canary_splitkv(vm):
+    # every unit split (fewer units than SMs, 66 key tiles with a ragged last one):
+    # output and workspace between guards
+    import torch
+    w = _ragged().with_(cached_frames=131)
+    wts = workload.layer_weights(w)
+    act = workload.batch_activations(w)
+    cache = torch.zeros(w.batch, w.n_kv, 224, dtype=torch.bfloat16, device="cuda")
+    gpu_fill_window(vm, w, to_dev(act["x"]), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache)
+    need = vm.vmla_chunk_attention_splitkv_workspace_bytes(w.batch, w.n_q, w.heads, w.n_kv)
+    assert need > 0 and need % 2 == 0
+    wbuf, ws = guarded(need // 2)
+    buf, out = guarded(w.batch, w.n_q, w.heads, 128)
+    vm.vmla_chunk_attention_splitkv(to_dev(act["q"]), to_dev(act["q_rope"]), to_dev(wts["w_uk"]),
+                                    to_dev(wts["w_uv"]), cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE, out,
+                                    workspace=ws)
+    vm.vmla_get_device_status()
+    assert_guards(buf, "splitkv output")
+    assert_guards(wbuf, "splitkv workspace")
