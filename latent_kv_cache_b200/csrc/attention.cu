@@ -772,18 +772,21 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         // this part is the last of its unit (it then merges all parts).
         bool merge = false, emit = true;
         int slot0 = 0;
+        // Partial O_lat layout: float4 (slot, half, 32-column group c, quarter q4,
+        // row), so that each warp access is one contiguous 512 B run.
+        auto part4 = [&](int slot, int c, int q4) -> float4* {
+          return reinterpret_cast<float4*>(p.ws_o) + ((((int64_t)slot * 2 + t.half) * C::kNb + c) * 8 + q4) * kBM + t.r;
+        };
         if (split > 1) {
           slot0 = (unit - p.n_full) * split;
-          float* wo = p.ws_o + ((int64_t)(slot0 + part) * kBM + t.r) * kDcT + (kDcT / 2) * t.half;
 #pragma unroll
           for (int c = 0; c < C::kNb; ++c) {  // this half's d_c/2 columns, 32 at a time
             tmem_ld32(t.t_row + kTmemO + (kDcT / 2) * t.half + 32 * c, v);
             tmem_ld_wait();
-            float4* dst = reinterpret_cast<float4*>(wo + 32 * c);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+              *part4(slot0 + part, c, q4) = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                                        __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
           }
           if (t.half == 0) {
             float2* ml = reinterpret_cast<float2*>(p.ws_ml) + (int64_t)(slot0 + part) * kBM + t.r;
@@ -832,12 +835,13 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
               for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(v[e]) * w_own;
               for (int r2 = 0; r2 < split; ++r2) {
                 if (r2 == part) continue;
-                const float4* src = reinterpret_cast<const float4*>(
-                    p.ws_o + ((int64_t)(slot0 + r2) * kBM + t.r) * kDcT + (kDcT / 2) * t.half + 32 * c);
                 const float w2 = exp2f(__ldcg(&ml[(int64_t)r2 * kBM].x) - m_tot);
+                float4 fs[8];
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) fs[q4] = __ldcg(part4(slot0 + r2, c, q4));
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
-                  const float4 f = __ldcg(src + q4);
+                  const float4 f = fs[q4];
                   acc[4 * q4] = fmaf(f.x, w2, acc[4 * q4]);
                   acc[4 * q4 + 1] = fmaf(f.y, w2, acc[4 * q4 + 1]);
                   acc[4 * q4 + 2] = fmaf(f.z, w2, acc[4 * q4 + 2]);
