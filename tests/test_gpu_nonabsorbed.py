@@ -144,3 +144,29 @@ def test_nonabsorbed_1080p_sampled(vm):
     ref = oracle.chunk_attention(act["q"], act["q_rope"], wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv, w.chunk_t0,
                                  w.grid_h, w.grid_w, SCALE, rows=rows)
     assert_close(to_f64(out)[:, rows], ref, "nonabsorbed 1080p")
+
+
+@pytest.mark.parametrize("name", ["tiny", "480p"])
+def test_dense_on_materialised_latent_equals_latent_attention(vm, name):
+    """Cross-check of the two layouts: with zero rope queries, the latent attention
+    over the cache equals dense per-head attention over the keys c.W_UK_h^T and
+    values c.W_UV_h^T that k_materialize_kv writes from the same cache."""
+    import torch
+    w = workload.CONFIGS[name]
+    wts = workload.layer_weights(w)
+    act = workload.batch_activations(w)
+    cache = torch.zeros(w.batch, w.n_kv, 224, dtype=torch.bfloat16, device="cuda")
+    gpu_fill_window(vm, w, to_dev(act["x"]), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache)
+    q = to_dev(act["q"])
+    qr0 = torch.zeros(w.batch, w.n_q, w.heads, 32, dtype=torch.bfloat16, device="cuda")
+    wuk, wuv = to_dev(wts["w_uk"]), to_dev(wts["w_uv"])
+    out_l = torch.empty(w.batch, w.n_q, w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_chunk_attention(q, qr0, wuk, wuv, cache, w.n_kv, w.chunk_t0, w.grid_h, w.grid_w, SCALE, out_l)
+    kv = torch.empty(w.batch, w.n_kv, 2 * w.heads, 128, dtype=torch.bfloat16, device="cuda")
+    vm.vmla_materialize_kv(wuk, wuv, cache, w.n_kv, kv)
+    k = kv[:, :, :w.heads].contiguous()
+    v = kv[:, :, w.heads:].contiguous()
+    out_d = torch.empty_like(out_l)
+    vm.vmla_dense_attention(q, k, v, SCALE, out_d)
+    vm.vmla_get_device_status()
+    assert_close(to_f64(out_l), to_f64(out_d), f"{name}: latent vs dense on materialised K/V")
