@@ -45,6 +45,26 @@ def test_bench_tiny_line():
     assert a["bound"] == "alu" and 0 < a["frac"] < 1.5
     assert b["dense"]["ms"] > 0 and b["nonabsorbed"]["ms_total"] > 0
     assert set(b["dc_sweep"]) == {"64", "128", "192", "256"}
+    assert b["splitkv"]["ms"] > 0 and b["splitkv"]["workspace_bytes"] == 0  # 5 key tiles: no split
+    assert "chunk_480p" not in b and "other_workloads" not in b            # 480P run only
+
+
+def test_bench_default_480p_line():
+    # the default workload, short: the per-chunk schedules, the sustained loop and the
+    # batch-8 / 1080P figures are in the line
+    b = _run("--steps", "2", "--warmup", "3", "--no-cpu-baseline", "--chunk-replays", "2")
+    assert b["config"]["workload"].startswith("480p")
+    assert b["roofline"]["frac"] > 0.5
+    c = b["chunk_480p"]
+    for k in ("nonabsorbed", "nonabsorbed_reuse", "dense"):
+        assert c[k]["ms_per_chunk"] > 0, k
+    assert c["nonabsorbed_reuse"]["transient_kv_bytes"] < c["nonabsorbed"]["transient_kv_bytes"]
+    s = c["sustained"]
+    assert s["seconds"] >= 2.0 and s["attention_tflops"] > 0
+    for name in ("480p_b8", "1080p"):
+        o = b["other_workloads"][name]
+        assert o["attention"]["ms"] > 0 and o["dense"]["ms"] > 0 and o["attention_splitkv"]["ms"] > 0
+    assert b["other_workloads"]["1080p"]["attention_splitkv"]["workspace_bytes"] > 0
 
 
 def test_bench_reference_arm_line():
