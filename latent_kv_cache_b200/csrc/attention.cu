@@ -11,12 +11,14 @@
 //
 // One CTA = one 128-query tile of one head of one sample; in the latent kernel heads
 // are the fastest grid index so the 12 CTAs that read the same cache tiles run
-// together and share them through L2 (the per-head dense and materialised kernels
-// put query tiles fastest instead).  Warp roles (320 threads):
+// together and share them through L2 (the per-head dense and materialised kernels,
+// further below, put query tiles fastest instead).  Warp roles (320 threads):
 //   warp 0      TMA producer: prologue operands, then key tiles into a ring.
 //   warp 1      TMEM allocation and the single MMA-issuing thread.
-//   warps 2..9  two softmax warpgroups; a thread owns one query row (= TMEM
-//               lane) and one half of the columns of every score tile.
+//   warps 2..9  two softmax warpgroups; in the latent kernel a thread owns one
+//               query row (= TMEM lane) and one half of the columns of every
+//               score tile (the per-head kernels give each warpgroup whole rows
+//               of every other key tile instead).
 //
 // The latent kernel is a template over the content width d_c (64, 128, 192 or
 // 256; the rope key stays 32 wide).  Its query operand Qa = [q_abs ; RoPE(q_r)]
@@ -47,15 +49,11 @@ constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kBM = 128;                          // queries per tile
 constexpr uint32_t kTmemCols = 512;
 
-// Kernel variants: latent chunk attention with W_UK absorbed (kKindMla), the dense
-// per-head baseline (kKindDense), and attention over per-head keys/values
-// materialised from the latent cache (kKindMat: content keys and values from a
-// [B, n_kv, 2H, 128] buffer, the rope key straight from the latent cache).
-enum Kind : int { kKindMla = 0, kKindDense = 1, kKindMat = 2 };
-
-// Per-variant configuration (kDcT: content width of the latent variant).
-template <int kKind, int kDcT = kDc>
-struct Cfg;
+// Per-head kernels (two-slot, below): the dense baseline (kKindDense) and attention
+// over per-head keys/values materialised from the latent cache (kKindMat: content
+// keys and values from a [B, n_kv, 2H, 128] buffer, the rope key straight from the
+// latent cache).
+enum Kind : int { kKindDense = 1, kKindMat = 2 };
 
 // MLA: the Qa operand (128 x (d_c + 32) bf16) sits in shared memory (SS MMAs for
 // the scores): O (d_c) + two 128-key S buffers (256) + Qa in TMEM would exceed
@@ -63,7 +61,7 @@ struct Cfg;
 // (a K = 16 tcgen05.mma takes at least ~93 cycles, so narrower N loses).
 // The ring is as deep as shared memory allows: 6, 4, 3, 2 stages.
 template <int kDcT>
-struct Cfg<kKindMla, kDcT> {
+struct Cfg {
   static_assert(kDcT == 64 || kDcT == 128 || kDcT == 192 || kDcT == 256, "d_c");
   static constexpr int kNb = kDcT / 64;                          // 128B-swizzled content blocks
   static constexpr int kBN = 128;                                // keys per tile
@@ -82,39 +80,12 @@ struct Cfg<kKindMla, kDcT> {
   static constexpr int kNbX = kParts == 3 ? kNb / 2 : kNb;  // content blocks in part X
 };
 
-// Dense: Q (64 cells of bf16 pairs) lives in TMEM; scores are TS MMAs.
-template <int kDcT>
-struct Cfg<kKindDense, kDcT> {
-  static constexpr int kBN = 128;
-  static constexpr int kStages = 3;
-  static constexpr uint32_t kBlkRows = 128 * 128;
-  static constexpr uint32_t kStage = 4 * kBlkRows;            // [K: 2 blocks | V: 2 blocks] = 65536
-  static constexpr uint32_t kQaBytes = 0;
-  static constexpr int kOCols = kDh;
-  static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
-  static constexpr int kParts = 1;
-};
-
-// Materialised keys/values: Q = [q_h ; RoPE(q_r)] (80 cells) in TMEM; key tile =
-// [content 128 ; rope 32], value tile 128.
-template <int kDcT>
-struct Cfg<kKindMat, kDcT> {
-  static constexpr int kBN = 128;
-  static constexpr int kStages = 3;
-  static constexpr uint32_t kBlkRows = 128 * 128;
-  static constexpr uint32_t kStage = 4 * kBlkRows + 128 * 64;  // [K: 2 | V: 2 blocks | k_r] = 73728
-  static constexpr uint32_t kQaBytes = 0;
-  static constexpr int kOCols = kDh;
-  static constexpr uint32_t kTmemS0 = 128, kTmemS1 = 256, kTmemQ = 384;
-  static constexpr int kParts = 1;
-};
-
 constexpr uint32_t kBlk128 = 128 * 128;  // 128 rows x 128 B: prologue / epilogue operand blocks
 constexpr uint32_t kTmemO = 0;
 
-template <int kKind, int kDcT = kDc>
+template <int kDcT>
 struct Layout {
-  using C = Cfg<kKind, kDcT>;
+  using C = Cfg<kDcT>;
   static constexpr uint32_t kRingOff = C::kQaBytes;
   static constexpr uint32_t kBarOff = kRingOff + C::kStages * C::kStage;
   static constexpr uint32_t kRedOff = kBarOff + 512;
@@ -128,7 +99,7 @@ struct Layout {
 // 0-1; the epilogue's W_UV_h (d_c/64 blocks) is one ring item.
 template <int kDcT>
 constexpr bool mla_fits() {
-  using C = Cfg<kKindMla, kDcT>;
+  using C = Cfg<kDcT>;
   return (2 + C::kNb) * kBlk128 <= 2 * C::kStage && C::kNb * kBlk128 <= C::kStage && C::kStages >= 2 &&
          kDcT + 256 <= (int)kTmemCols && kDcT / 2 <= 128;
 }
@@ -155,20 +126,9 @@ struct ChunkMaps {
   CUtensorMap kr;   // [B, n_kv, d_c + 32]  box (32, 128, 1), 64B swizzle (rope key, x = d_c)
 };
 
-struct DenseMaps {
-  CUtensorMap k;  // [B, Nk, H, 128] box (64, 1, 128, 1)
-  CUtensorMap v;  // [B, Nk, H, 128]
-};
-
-struct MatMaps {
-  CUtensorMap k;   // [B, n_kv, 2H, 128] box (64, 1, 128, 1): heads [0, H) keys, [H, 2H) values
-  CUtensorMap v;   // same tensor (values addressed at head H + h)
-  CUtensorMap kr;  // latent cache [B, n_kv, 224] box (32, 128, 1), 64B swizzle (rope key, x = 192)
-};
-
 struct AttnParams {
-  const uint16_t* q;       // dense: queries are read directly into tensor memory
-  const uint16_t* q_rope;  // MLA only
+  const uint16_t* q;
+  const uint16_t* q_rope;  // latent and materialised kernels
   uint16_t* out;
   int* status;
   uint64_t wait_limit_ns;
@@ -257,22 +217,22 @@ __device__ __forceinline__ bool exchange(const SoftmaxThread& t, uint32_t bars, 
 // Softmax step for key tile j.  Returns false on abort.
 // j: tile index within this CTA's key range (barrier phases); jabs: the tile's
 // index in the key sequence (masking of keys >= n_kv).
-template <int kKind, int kDcT>
+template <int kDcT>
 __device__ __forceinline__ bool softmax_tile(int j, int jabs, uint32_t bars, const SoftmaxThread& t,
                                              const AttnParams& p, const WaitCtl& ctl,
                                              float& m_run, float& l_part) {
-  using C = Cfg<kKind, kDcT>;
-  constexpr int kW = C::kBN / 2;  // score columns per thread (48 or 64)
+  using C = Cfg<kDcT>;
+  constexpr int kW = C::kBN / 2;  // score columns per thread
   const int sb = j & 1;
   if (!warp_wait(bar_addr(bars, B_SF0 + sb), (j >> 1) & 1, ctl)) return false;
   tc_fence_after();
   const uint32_t sbase = sb ? C::kTmemS1 : C::kTmemS0;
+  static_assert(kW == 64, "64 score columns per thread");
   float s[kW];
   {
-    uint32_t ra[32], rb[kW - 32];
+    uint32_t ra[32], rb[32];
     tmem_ld32(t.t_row + sbase + kW * t.half, ra);
-    if constexpr (kW - 32 == 16) tmem_ld16(t.t_row + sbase + kW * t.half + 32, rb);
-    else tmem_ld32(t.t_row + sbase + kW * t.half + 32, rb);
+    tmem_ld32(t.t_row + sbase + kW * t.half + 32, rb);
     tmem_ld_wait();
 #pragma unroll
     for (int e = 0; e < 32; ++e) s[e] = __uint_as_float(ra[e]);
@@ -315,13 +275,7 @@ __device__ __forceinline__ bool softmax_tile(int j, int jabs, uint32_t bars, con
     pk[e] = pack_bf16x2(p0, p1);
   }
   // P (bf16 pairs) over the first kBN/2 cells of the S buffer: this half's kW/2 cells.
-  const uint32_t pcol = t.t_row + sbase + (kW / 2) * t.half;
-  if constexpr (kW / 2 == 24) {
-    tmem_st16(pcol, pk);
-    tmem_st8(pcol + 16, pk + 16);
-  } else {
-    tmem_st32(pcol, pk);
-  }
+  tmem_st32(t.t_row + sbase + (kW / 2) * t.half, pk);
   sum[0] += sum[4]; sum[1] += sum[5]; sum[2] += sum[6]; sum[3] += sum[7];
   sum[0] += sum[2]; sum[1] += sum[3];
   l_part = l_part * alpha + (sum[0] + sum[1]);
@@ -383,16 +337,14 @@ __device__ __forceinline__ void rope_query(const AttnParams& p, const RopeTable*
 }
 
 // ---------------------------------------------------------------------------
-// The attention kernel.  kMla: latent chunk attention (absorbed W_UK, [c ; k_r]
-// tiles, W_UV epilogue) with content width kDcT; kMat: attention over
-// materialised per-head keys/values; otherwise the dense per-head baseline.
+// The latent kernel: chunk attention with W_UK absorbed into the queries,
+// [c ; k_r] key tiles that also serve as the values, and the W_UV epilogue, for
+// content width kDcT.
 // ---------------------------------------------------------------------------
-template <int kKind, int kDcT, class Maps>
-__device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p, const RopeTable* tab) {
-  constexpr bool kMla = kKind == kKindMla;
-  constexpr bool kMat = kKind == kKindMat;
-  using C = Cfg<kKind, kDcT>;
-  using L = Layout<kKind, kDcT>;
+template <int kDcT>
+__device__ __forceinline__ void attn_body(const ChunkMaps& maps, const AttnParams& p, const RopeTable* tab) {
+  using C = Cfg<kDcT>;
+  using L = Layout<kDcT>;
   constexpr int kBN = C::kBN;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kStage = C::kStage;
@@ -404,7 +356,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     return;
   }
   uint8_t* smem = smem_raw + pad;
-  const uint32_t qa = smem_u32(smem);    // MLA: Qa tile (d_c/64 SW128 blocks + SW64 rope block)
+  const uint32_t qa = smem_u32(smem);    // Qa tile (d_c/64 SW128 blocks + SW64 rope block)
   const uint32_t st0 = qa + L::kRingOff; // ring stage s at st0 + s * kStage
   const uint32_t bars = qa + L::kBarOff;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * B_COUNT);
@@ -415,14 +367,12 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Grid order.  Latent kernel: heads fastest, so the 12 head-CTAs of a query
-  // tile, which read the same cache tiles, run together.  Dense and materialised
-  // kernels: query tiles fastest, so the CTAs that run together share one head's
-  // key/value tiles and each head's keys and values cross HBM about once.
+  // Grid order: heads fastest, so the 12 head-CTAs of a query tile, which read
+  // the same cache tiles, run together.  1-D grid: whole units first, then the
+  // parts of the split units.
   const int n_qt = (p.n_q + kBM - 1) / kBM;
-  int h, q0, b, unit = 0, part = 0, split = 1;
-  if constexpr (kMla) {
-    // 1-D grid: whole units first, then the parts of the split units.
+  int unit = 0, part = 0, split = 1;
+  {
     const int u = (int)blockIdx.x;
     if (u < p.n_full) {
       unit = u;
@@ -431,15 +381,11 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       part = (u - p.n_full) % p.split;
       split = p.split;
     }
-    const int per_b = n_qt * p.heads;
-    b = unit / per_b;
-    h = (unit % per_b) % p.heads;
-    q0 = ((unit % per_b) / p.heads) * kBM;
-  } else {
-    h = (int)(blockIdx.x / n_qt);
-    q0 = (int)(blockIdx.x % n_qt) * kBM;
-    b = (int)blockIdx.y;
   }
+  const int per_b = n_qt * p.heads;
+  const int b = unit / per_b;
+  const int h = (unit % per_b) % p.heads;
+  const int q0 = ((unit % per_b) / p.heads) * kBM;
   // This CTA's key tiles: [kt0, kt0 + n_tiles) of the n_kv_tiles tiles.
   const int kt0 = (int)((int64_t)part * p.n_kv_tiles / split);
   const int n_tiles = (int)((int64_t)(part + 1) * p.n_kv_tiles / split) - kt0;
@@ -488,30 +434,24 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
 #pragma unroll
         for (int s = 0; s < kStages; ++s) last_use[x][s] = -1;
       bool ok = true;
-      if constexpr (kMla) {
-        tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.wuk);
-        tma_prefetch_desc(&maps.wuv);
-        tma_prefetch_desc(&maps.c);
-        tma_prefetch_desc(&maps.kr);
-        // Prologue operands borrow ring stages 0-1: q tile (2 blocks) then W_UK_h (d_c/64 blocks).
-        mbar_arrive_expect_tx(bar_addr(bars, B_PRO), (2 + C::kNb) * kBlk128);
-        tma_load_4d(st0, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
-        tma_load_4d(st0 + kBlk128, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.wuk);
+      tma_prefetch_desc(&maps.wuv);
+      tma_prefetch_desc(&maps.c);
+      tma_prefetch_desc(&maps.kr);
+      // Prologue operands borrow ring stages 0-1: q tile (2 blocks) then W_UK_h (d_c/64 blocks).
+      mbar_arrive_expect_tx(bar_addr(bars, B_PRO), (2 + C::kNb) * kBlk128);
+      tma_load_4d(st0, &maps.q, bar_addr(bars, B_PRO), 0, h, q0, b);
+      tma_load_4d(st0 + kBlk128, &maps.q, bar_addr(bars, B_PRO), 64, h, q0, b);
 #pragma unroll
-        for (int i = 0; i < C::kNb; ++i)
-          tma_load_2d(st0 + (2 + i) * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 64 * i, h * kDh);
-      } else {
-        tma_prefetch_desc(&maps.k);
-        tma_prefetch_desc(&maps.v);
-        if constexpr (kMat) tma_prefetch_desc(&maps.kr);
-      }
-      // MLA: n_tiles key tiles, then the W_UV_h blocks as one more ring item.
-      const int n_items = kMla ? n_tiles + 1 : n_tiles;
+      for (int i = 0; i < C::kNb; ++i)
+        tma_load_2d(st0 + (2 + i) * kBlk128, &maps.wuk, bar_addr(bars, B_PRO), 64 * i, h * kDh);
+      // n_tiles key tiles, then the W_UV_h blocks as one more ring item.
+      const int n_items = n_tiles + 1;
       for (int i = 0; ok && i < n_items; ++i) {
         const int st = i % kStages, use = i / kStages;
         const uint32_t sa = st0 + st * kStage;
-        if (use == 0 && kMla && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
+        if (use == 0 && st < 2) ok = mbar_wait(bar_addr(bars, B_QABS), 0, ctl, kDevTimeoutProducer);
         for (int x = 0; ok && x < kParts; ++x) {
           // Three-part stages: the W_UV item has no rope part (and is the stage's last use).
           if (kParts == 3 && x == 0 && i == n_tiles) continue;
@@ -520,34 +460,24 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
           if (!ok) break;
           const uint32_t fb = bar_addr(bars, B_KVF0 + x * kStages + st);
           const int kv0 = (kt0 + i) * kBN;
-          if constexpr (kMla) {
-            // part x: content blocks [blo, bhi) and (rope) the 64B-swizzled rope block
-            const int blo = kParts == 1 ? 0 : x == 2 ? C::kNbX : 0;
-            const int bhi = kParts == 1 ? C::kNb : x == 0 ? 0 : x == 1 ? C::kNbX : C::kNb;
-            const bool rope = kParts == 1 || x == 0;
-            if (i < n_tiles) {
-              mbar_arrive_expect_tx(fb, (bhi - blo) * C::kBlkRows + (rope ? 128u * 64u : 0u));
-              for (int blk = blo; blk < bhi; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
-              if (rope) tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
-            } else {
-              mbar_arrive_expect_tx(fb, (bhi - blo) * kBlk128);
-              for (int blk = blo; blk < bhi; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
-            }
+          // part x: content blocks [blo, bhi) and (rope) the 64B-swizzled rope block
+          const int blo = kParts == 1 ? 0 : x == 2 ? C::kNbX : 0;
+          const int bhi = kParts == 1 ? C::kNb : x == 0 ? 0 : x == 1 ? C::kNbX : C::kNb;
+          const bool rope = kParts == 1 || x == 0;
+          if (i < n_tiles) {
+            mbar_arrive_expect_tx(fb, (bhi - blo) * C::kBlkRows + (rope ? 128u * 64u : 0u));
+            for (int blk = blo; blk < bhi; ++blk) tma_load_3d(sa + blk * C::kBlkRows, &maps.c, fb, 64 * blk, kv0, b);
+            if (rope) tma_load_3d(sa + C::kNb * C::kBlkRows, &maps.kr, fb, kDcT, kv0, b);
           } else {
-            const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
-            mbar_arrive_expect_tx(fb, kStage);
-            tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
-            tma_load_4d(sa + C::kBlkRows, &maps.k, fb, 64, h, kv0, b);
-            tma_load_4d(sa + 2 * C::kBlkRows, &maps.v, fb, 0, hv, kv0, b);
-            tma_load_4d(sa + 3 * C::kBlkRows, &maps.v, fb, 64, hv, kv0, b);
-            if constexpr (kMat) tma_load_3d(sa + 4 * C::kBlkRows, &maps.kr, fb, kDc, kv0, b);
+            mbar_arrive_expect_tx(fb, (bhi - blo) * kBlk128);
+            for (int blk = blo; blk < bhi; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
           }
           last_use[x][st] = use;
         }
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits.
-        if (kMla) drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
+        drain_wait(bar_addr(bars, B_PRO), 0, p.wait_limit_ns, p.status);
         for (int x = 0; x < kParts; ++x)
           for (int s = 0; s < kStages; ++s)
             if (last_use[x][s] >= 0)
@@ -559,29 +489,26 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       // --------------------------------- MMA ----------------------------------
       constexpr uint32_t kIdS = idesc_bf16_f32(128, kBN, false, false);
       constexpr uint32_t kIdPv = idesc_bf16_f32(128, C::kOCols, false, true);
-      bool ok = true;
-      if constexpr (kMla) {
-        ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
-        if (ok) {
-          constexpr uint32_t kIdQabs = idesc_bf16_f32(128, kDcT, false, true);
-          tc_fence_after();
-          // q_abs = q_h . W_UK_h (M 128, N d_c, K 128): q K-major, W_UK MN-major.
+      bool ok = mbar_wait(bar_addr(bars, B_PRO), 0, ctl, kDevTimeoutMma);
+      if (ok) {
+        constexpr uint32_t kIdQabs = idesc_bf16_f32(128, kDcT, false, true);
+        tc_fence_after();
+        // q_abs = q_h . W_UK_h (M 128, N d_c, K 128): q K-major, W_UK MN-major.
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
-            const uint64_t bd = smem_desc(st0 + 2 * kBlk128 + k * 2048, kBlk128, 1024, kSw128);
-            umma_ss(tmem + kTmemO, a, bd, kIdQabs, k > 0);
-          }
-          umma_commit(bar_addr(bars, B_QABS));
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
+          const uint64_t bd = smem_desc(st0 + 2 * kBlk128 + k * 2048, kBlk128, 1024, kSw128);
+          umma_ss(tmem + kTmemO, a, bd, kIdQabs, k > 0);
         }
+        umma_commit(bar_addr(bars, B_QABS));
       }
       if (ok) ok = mbar_wait(bar_addr(bars, B_QA), 0, ctl, kDevTimeoutMma);
       auto issue_pv = [&](int jj) -> bool {
         if (!mbar_wait(bar_addr(bars, B_PF0 + (jj & 1)), (jj >> 1) & 1, ctl, kDevTimeoutMma))
           return false;
         tc_fence_after();
-        // V operand: the latent c blocks (MLA) or the V blocks (dense), MN-major.
-        const uint32_t sv = st0 + (jj % kStages) * kStage + (kMla ? 0u : 2 * C::kBlkRows);
+        // Value operand: the latent c blocks of the same stage, MN-major.
+        const uint32_t sv = st0 + (jj % kStages) * kStage;
         const uint32_t a_t = tmem + ((jj & 1) ? C::kTmemS1 : C::kTmemS0);
         if constexpr (C::kParts == 3) {
           // Two halves of the latent columns; part X of the stage is free after the
@@ -616,67 +543,53 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
         tc_fence_after();
         const uint32_t sa = st0 + st * kStage;
         const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
-        if constexpr (kMla) {
-          // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
-          // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
-          // share offsets.  With a stage in three parts the K steps run in the order
-          // R (the rope block), X, Y, each part waited for just before its steps,
-          // and R is released as soon as the scores are done.
-          constexpr int kCs = 4 * C::kNb;
-          constexpr int kCx = 4 * C::kNbX;  // content steps in part X
+        // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
+        // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
+        // share offsets.  With a stage in three parts the K steps run in the order
+        // R (the rope block), X, Y, each part waited for just before its steps,
+        // and R is released as soon as the scores are done.
+        constexpr int kCs = 4 * C::kNb;
+        constexpr int kCx = 4 * C::kNbX;  // content steps in part X
 #pragma unroll
-          for (int n = 0; n < kCs + 2; ++n) {
-            const int k = C::kParts == 3 ? (n < 2 ? kCs + n : n - 2) : n;
-            if (C::kParts == 3 && (n == 2 || n == 2 + kCx)) {  // (part R was waited for above)
-              const int x = n == 2 ? 1 : 2;
-              ok = mbar_wait(bar_addr(bars, B_KVF0 + x * kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            const uint32_t off = k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32;
-            const uint32_t sbo = k < kCs ? 1024 : 512;
-            const uint32_t lay = k < kCs ? kSw128 : kSw64;
-            umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, n > 0);
+        for (int n = 0; n < kCs + 2; ++n) {
+          const int k = C::kParts == 3 ? (n < 2 ? kCs + n : n - 2) : n;
+          if (C::kParts == 3 && (n == 2 || n == 2 + kCx)) {  // (part R was waited for above)
+            const int x = n == 2 ? 1 : 2;
+            ok = mbar_wait(bar_addr(bars, B_KVF0 + x * kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
+            if (!ok) break;
+            tc_fence_after();
           }
-          if (!ok) break;
-          if constexpr (C::kParts == 3) umma_commit(bar_addr(bars, B_KVE0 + st));  // R free once S is done
-        } else {
-          // S = Q . K^T with Q from TMEM: 8 steps over the 128B-swizzled content key
-          // blocks (+2 over the 64B-swizzled rope block for the materialised variant).
-          constexpr int kSteps = kMat ? 10 : 8;
-#pragma unroll
-          for (int k = 0; k < kSteps; ++k) {
-            const uint64_t bd = k < 8 ? smem_desc(sa + (k >> 2) * C::kBlkRows + (k & 3) * 32, 16, 1024, kSw128)
-                                      : smem_desc(sa + 4 * C::kBlkRows + (k - 8) * 32, 16, 512, kSw64);
-            umma_ts(d, tmem + C::kTmemQ + k * 8, bd, kIdS, k > 0);
-          }
+          const uint32_t off = k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32;
+          const uint32_t sbo = k < kCs ? 1024 : 512;
+          const uint32_t lay = k < kCs ? kSw128 : kSw64;
+          umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, n > 0);
         }
+        if (!ok) break;
+        if constexpr (C::kParts == 3) umma_commit(bar_addr(bars, B_KVE0 + st));  // R free once S is done
         umma_commit(bar_addr(bars, B_SF0 + (j & 1)));
         if (j >= 1) ok = issue_pv(j - 1);
       }
       if (ok) ok = issue_pv(n_tiles - 1);
-      if constexpr (kMla) {
-        if (ok) {
-          constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
-          const int sw = n_tiles % kStages;
-          // W_UV_h blocks: the whole stage, or parts X and Y of a three-part stage.
-          const int ph = (n_tiles / kStages) & 1;
-          ok = (C::kParts == 1
-                    ? mbar_wait(bar_addr(bars, B_KVF0 + sw), ph, ctl, kDevTimeoutMma)
-                    : mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), ph, ctl, kDevTimeoutMma) &&
-                          mbar_wait(bar_addr(bars, B_KVF0 + 2 * kStages + sw), ph, ctl, kDevTimeoutMma)) &&
-               mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
-          if (ok && !*skip_flag) {  // (a part of a split unit that does not merge skips it)
-            tc_fence_after();
-            const uint32_t wb = st0 + sw * kStage;
-            // out = O_lat/l . W_UV_h^T (M 128, N 128, K d_c): A from TMEM, W_UV K-major.
+      if (ok) {
+        constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
+        const int sw = n_tiles % kStages;
+        // W_UV_h blocks: the whole stage, or parts X and Y of a three-part stage.
+        const int ph = (n_tiles / kStages) & 1;
+        ok = (C::kParts == 1
+                  ? mbar_wait(bar_addr(bars, B_KVF0 + sw), ph, ctl, kDevTimeoutMma)
+                  : mbar_wait(bar_addr(bars, B_KVF0 + kStages + sw), ph, ctl, kDevTimeoutMma) &&
+                        mbar_wait(bar_addr(bars, B_KVF0 + 2 * kStages + sw), ph, ctl, kDevTimeoutMma)) &&
+             mbar_wait(bar_addr(bars, B_OA), 0, ctl, kDevTimeoutMma);
+        if (ok && !*skip_flag) {  // (a part of a split unit that does not merge skips it)
+          tc_fence_after();
+          const uint32_t wb = st0 + sw * kStage;
+          // out = O_lat/l . W_UV_h^T (M 128, N 128, K d_c): A from TMEM, W_UV K-major.
 #pragma unroll
-            for (int k = 0; k < kDcT / 16; ++k) {
-              const uint64_t bd = smem_desc(wb + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
-              umma_ts(tmem + C::kTmemS1, tmem + C::kTmemS0 + k * 8, bd, kIdOut, k > 0);
-            }
-            umma_commit(bar_addr(bars, B_OUT));
+          for (int k = 0; k < kDcT / 16; ++k) {
+            const uint64_t bd = smem_desc(wb + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
+            umma_ts(tmem + C::kTmemS1, tmem + C::kTmemS0 + k * 8, bd, kIdOut, k > 0);
           }
+          umma_commit(bar_addr(bars, B_OUT));
         }
       }
       if (!ok) {
@@ -693,63 +606,35 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     t.t_row = tmem + ((uint32_t)(t.qd * 32) << 16);
     t.red = red;
     const int qi = q0 + t.r;
-    bool ok = true;
-    if constexpr (kMla) {
-      ok = warp_wait(bar_addr(bars, B_QABS), 0, ctl);
-      if (ok) {
-        tc_fence_after();
-        // q_abs (fp32, TMEM) -> bf16 Qa tile in shared memory; this half: columns
-        // [d_c/2 half, +d_c/2).
-        uint32_t v[32];
-#pragma unroll
-        for (int c = 0; c < C::kNb; ++c) {
-          const int col = (kDcT / 2) * t.half + 32 * c;
-          tmem_ld32(t.t_row + kTmemO + col, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            st_sw128_chunk(smem + (col >> 6) * C::kBlkRows, t.r, ((col & 63) >> 3) + q4, pack8(v + 8 * q4, 1.0f));
-        }
-        if (t.half == 0) {
-          float qr[kDr];
-          rope_query(p, tab, b, qi, h, qr);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 w;
-            w.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
-            w.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
-            w.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
-            w.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
-            st_sw64_chunk(smem + C::kNb * C::kBlkRows, t.r, c, w);
-          }
-        }
-        fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
-      }
-    } else {
-      // Dense queries straight from global memory into the Q cells (bf16 pairs).
+    bool ok = warp_wait(bar_addr(bars, B_QABS), 0, ctl);
+    if (ok) {
+      tc_fence_after();
+      // q_abs (fp32, TMEM) -> bf16 Qa tile in shared memory; this half: columns
+      // [d_c/2 half, +d_c/2).
       uint32_t v[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = 0u;
-      if (qi < p.n_q) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.q + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh + 64 * t.half);
+      for (int c = 0; c < C::kNb; ++c) {
+        const int col = (kDcT / 2) * t.half + 32 * c;
+        tmem_ld32(t.t_row + kTmemO + col, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 u = __ldg(src + c);
-          v[4 * c + 0] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_sw128_chunk(smem + (col >> 6) * C::kBlkRows, t.r, ((col & 63) >> 3) + q4, pack8(v + 8 * q4, 1.0f));
+      }
+      if (t.half == 0) {
+        float qr[kDr];
+        rope_query(p, tab, b, qi, h, qr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 w;
+          w.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
+          w.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
+          w.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
+          w.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
+          st_sw64_chunk(smem + C::kNb * C::kBlkRows, t.r, c, w);
         }
       }
-      tmem_st32(t.t_row + C::kTmemQ + 32 * t.half, v);
-      if constexpr (kMat) {
-        if (t.half == 0) {
-          float qr[kDr];
-          rope_query(p, tab, b, qi, h, qr);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(qr[2 * e], qr[2 * e + 1]);
-          tmem_st16(t.t_row + C::kTmemQ + 64, pk);
-        }
-      }
+      fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
     }
     if (ok) {
       tmem_st_wait();
@@ -758,7 +643,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
     }
     float m_run = -INFINITY, l_part = 0.0f;
     for (int j = 0; ok && j < n_tiles; ++j)
-      ok = softmax_tile<kKind, kDcT>(j, kt0 + j, bars, t, p, ctl, m_run, l_part);
+      ok = softmax_tile<kDcT>(j, kt0 + j, bars, t, p, ctl, m_run, l_part);
     float l_other = 0.0f;
     if (ok) ok = exchange(t, bars, n_tiles, l_part, l_other, ctl);
     if (ok) ok = warp_wait(bar_addr(bars, B_PV), (n_tiles - 1) & 1, ctl);
@@ -767,7 +652,7 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
       const float inv_l = 1.0f / (l_part + l_other);
       uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
       uint32_t v[32];
-      if constexpr (kMla) {
+      {
         // Split unit: write this part's partial, count it in, and find out whether
         // this part is the last of its unit (it then merges all parts).
         bool merge = false, emit = true;
@@ -874,17 +759,6 @@ __device__ __forceinline__ void attn_body(const Maps& maps, const AttnParams& p,
             }
           }
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(t.t_row + kTmemO + 64 * t.half + 32 * c, v);
-          tmem_ld_wait();
-          if (qi < p.n_q) {
-            uint4* dst = reinterpret_cast<uint4*>(out_row + 64 * t.half + 32 * c);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = pack8(v + 8 * q4, inv_l);
-          }
-        }
       }
     }
   }
@@ -902,18 +776,403 @@ template <int kDcT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_chunk_attn(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
                  const __grid_constant__ RopeTable tab) {
-  attn_body<kKindMla, kDcT>(maps, p, &tab);
+  attn_body<kDcT>(maps, p, &tab);
+}
+
+// ---------------------------------------------------------------------------
+// Two-slot kernels for the per-head attention (dense baseline and materialised
+// keys/values).  One CTA is one 128-query tile of one head of one sample, and
+// its two softmax warpgroups do not split each score tile by columns as the
+// latent kernel's do: warpgroup w ("slot" w) owns whole rows of every other key tile (tiles
+// j = w, w + 2, ...), with its own score buffer S_w, its own output accumulator
+// O_w and its own running max and sum; the two partial results are merged once,
+// after the last tile.  So no per-tile exchange of row maxima is needed, and
+// while one slot runs the exponentials of its tile the tensor pipe computes the
+// other slot's scores and P.V products.  The query tile sits in shared memory
+// (SS score MMAs), since tensor memory is taken up by the two S buffers and the
+// two accumulators:
+//   [0, 128) S_0 (P_0 as bf16 pairs over its first 64 cells)   [128, 256) S_1
+//   [256, 384) O_0                                              [384, 512) O_1
+// The MMA thread issues, after S_0(0) and S_1(1):
+//   PV_0(0), S_0(2), PV_1(1), S_1(3), PV_0(2), S_0(4), ...
+// so each slot's next score tile is queued right behind its own P.V product and
+// a slot has the other slot's two MMA groups of time for its softmax.
+// Key tiles (and the materialised variant's rope keys) and value tiles stream
+// through two rings: a key stage is released when its scores are done, a value
+// stage when its P.V product is.
+// ---------------------------------------------------------------------------
+template <int kKind>
+struct PpCfg {
+  static constexpr bool kMat = kKind == kKindMat;
+  static constexpr int kKSteps = kMat ? 10 : 8;                          // score K steps of 16
+  static constexpr uint32_t kQBytes = 2 * kBlk128 + (kMat ? 128u * 64u : 0u);  // q_h (+ rope block)
+  static constexpr uint32_t kKStage = kQBytes;                           // key tile: same block structure
+  static constexpr uint32_t kVStage = 2 * kBlk128;
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = kMat ? 2 : 3;
+  static constexpr uint32_t kKOff = kQBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kKStage;
+  static constexpr uint32_t kBarOff = kVOff + kVStages * kVStage;
+  static constexpr uint32_t kRedOff = kBarOff + 512;
+  static constexpr uint32_t kUsed = kRedOff + 2 * 2 * 128 * 4;           // (m, l) of both slots
+  static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
+  static constexpr uint32_t kMaxPad = kBytes - kUsed;
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
+  static_assert(kUsed + 512 <= 232448, "shared memory (with at least 512 B of alignment slack)");
+};
+
+enum PpBar {
+  P_Q = 0, P_QR,
+  P_KF0, P_KE0 = P_KF0 + 3, P_VF0 = P_KE0 + 3, P_VE0 = P_VF0 + 3,
+  P_SF0 = P_VE0 + 3, P_SF1, P_PF0, P_PF1, P_PV0, P_PV1,
+  P_MRG, P_DRAIN,
+  P_COUNT
+};
+static_assert(P_COUNT * 8 + 16 <= 512, "barrier area");
+
+struct PpMaps {
+  CUtensorMap q;   // [B, Nq, H, 128] box (64, 1, 128, 1), 128B swizzle
+  CUtensorMap k;   // dense: [B, Nk, H, 128]; materialised: [B, n_kv, 2H, 128] (keys at heads [0, H))
+  CUtensorMap v;   // dense: [B, Nk, H, 128]; materialised: same tensor (values at head H + h)
+  CUtensorMap kr;  // materialised only: latent cache [B, n_kv, 224] box (32, 128, 1), 64B swizzle
+};
+
+template <int kKind>
+__device__ __forceinline__ void pp_body(const PpMaps& maps, const AttnParams& p, const RopeTable* tab) {
+  using C = PpCfg<kKind>;
+  constexpr bool kMat = C::kMat;
+  constexpr int kKS = C::kKStages, kVS = C::kVStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
+  const uint32_t pad = (uint32_t)(((raw + 1023) & ~uintptr_t(1023)) - raw);
+  if (pad > C::kMaxPad) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kDevSmemMisaligned);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t qs = smem_u32(smem);  // query tile
+  const uint32_t ks0 = qs + C::kKOff;  // key stage s at ks0 + s * kKStage
+  const uint32_t vs0 = qs + C::kVOff;  // value stage s at vs0 + s * kVStage
+  const uint32_t bars = qs + C::kBarOff;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * P_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* red = reinterpret_cast<float*>(smem + C::kRedOff);  // [slot][m | l][128 rows]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_qt = (p.n_q + kBM - 1) / kBM;
+  const int h = (int)(blockIdx.x / n_qt);  // query tiles fastest: co-running CTAs share a head's K/V
+  const int q0 = (int)(blockIdx.x % n_qt) * kBM;
+  const int b = (int)blockIdx.y;
+  const int n_tiles = p.n_kv_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_addr(bars, P_Q), 1);
+    mbar_init(bar_addr(bars, P_QR), 128);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(bar_addr(bars, P_KF0 + s), 1);
+      mbar_init(bar_addr(bars, P_KE0 + s), 1);
+      mbar_init(bar_addr(bars, P_VF0 + s), 1);
+      mbar_init(bar_addr(bars, P_VE0 + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_addr(bars, P_SF0 + s), 1);
+      mbar_init(bar_addr(bars, P_PF0 + s), 128);
+      mbar_init(bar_addr(bars, P_PV0 + s), 1);
+    }
+    mbar_init(bar_addr(bars, P_MRG), kSoftmaxThreads);
+    mbar_init(bar_addr(bars, P_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------- producer -------------------------------
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      if constexpr (kMat) tma_prefetch_desc(&maps.kr);
+      mbar_arrive_expect_tx(bar_addr(bars, P_Q), 2 * kBlk128);
+      tma_load_4d(qs, &maps.q, bar_addr(bars, P_Q), 0, h, q0, b);
+      tma_load_4d(qs + kBlk128, &maps.q, bar_addr(bars, P_Q), 64, h, q0, b);
+      int k_last[kKS], v_last[kVS];
+#pragma unroll
+      for (int s = 0; s < kKS; ++s) k_last[s] = -1;
+#pragma unroll
+      for (int s = 0; s < kVS; ++s) v_last[s] = -1;
+      auto load_k = [&](int j) -> bool {
+        const int st = j % kKS, use = j / kKS;
+        if (use > 0 && !mbar_wait(bar_addr(bars, P_KE0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer))
+          return false;
+        const uint32_t fb = bar_addr(bars, P_KF0 + st), sa = ks0 + st * C::kKStage;
+        const int kv0 = j * 128;
+        mbar_arrive_expect_tx(fb, C::kKStage);
+        tma_load_4d(sa, &maps.k, fb, 0, h, kv0, b);
+        tma_load_4d(sa + kBlk128, &maps.k, fb, 64, h, kv0, b);
+        if constexpr (kMat) tma_load_3d(sa + 2 * kBlk128, &maps.kr, fb, kDc, kv0, b);
+        k_last[st] = use;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j % kVS, use = j / kVS;
+        if (use > 0 && !mbar_wait(bar_addr(bars, P_VE0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer))
+          return false;
+        const uint32_t fb = bar_addr(bars, P_VF0 + st), sa = vs0 + st * C::kVStage;
+        const int kv0 = j * 128;
+        const int hv = kMat ? p.heads + h : h;  // materialised values follow the H key heads
+        mbar_arrive_expect_tx(fb, C::kVStage);
+        tma_load_4d(sa, &maps.v, fb, 0, hv, kv0, b);
+        tma_load_4d(sa + kBlk128, &maps.v, fb, 64, hv, kv0, b);
+        v_last[st] = use;
+        return true;
+      };
+      // In the order the MMA thread consumes them: K0, K1, then V_j, K_{j+2}.
+      bool ok = load_k(0);
+      if (ok && n_tiles > 1) ok = load_k(1);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        ok = load_v(j);
+        if (ok && j + 2 < n_tiles) ok = load_k(j + 2);
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA exits.
+        drain_wait(bar_addr(bars, P_Q), 0, p.wait_limit_ns, p.status);
+        for (int s = 0; s < kKS; ++s)
+          if (k_last[s] >= 0) drain_wait(bar_addr(bars, P_KF0 + s), k_last[s] & 1, p.wait_limit_ns, p.status);
+        for (int s = 0; s < kVS; ++s)
+          if (v_last[s] >= 0) drain_wait(bar_addr(bars, P_VF0 + s), v_last[s] & 1, p.wait_limit_ns, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------- MMA ----------------------------------
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPv = idesc_bf16_f32(128, kDh, false, true);
+      bool ok = mbar_wait(bar_addr(bars, P_Q), 0, ctl, kDevTimeoutMma);
+      if (ok && kMat) ok = mbar_wait(bar_addr(bars, P_QR), 0, ctl, kDevTimeoutMma);
+      // S_w = Q . K_j^T (w = j & 1): 8 steps over the 128B-swizzled blocks (+2 over
+      // the 64B-swizzled rope block); the query and key tiles share offsets.
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % kKS;
+        if (!mbar_wait(bar_addr(bars, P_KF0 + st), (j / kKS) & 1, ctl, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t sa = ks0 + st * C::kKStage;
+        const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+        for (int k = 0; k < C::kKSteps; ++k) {
+          const uint32_t off = k < 8 ? (k >> 2) * kBlk128 + (k & 3) * 32 : 2 * kBlk128 + (k - 8) * 32;
+          const uint32_t sbo = k < 8 ? 1024 : 512;
+          const uint32_t lay = k < 8 ? kSw128 : kSw64;
+          umma_ss(d, smem_desc(qs + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
+        }
+        umma_commit(bar_addr(bars, P_SF0 + (j & 1)));
+        umma_commit(bar_addr(bars, P_KE0 + st));
+        return true;
+      };
+      // O_w += P_w . V_j: P from TMEM (bf16 pairs over S_w), V MN-major.
+      auto issue_pv = [&](int j) -> bool {
+        const int w = j & 1, st = j % kVS;
+        if (!mbar_wait(bar_addr(bars, P_PF0 + w), (j >> 1) & 1, ctl, kDevTimeoutMma)) return false;
+        if (!mbar_wait(bar_addr(bars, P_VF0 + st), (j / kVS) & 1, ctl, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t sv = vs0 + st * C::kVStage;
+        const uint32_t a_t = tmem + (w ? C::kTmemS1 : C::kTmemS0);
+        const uint32_t d = tmem + (w ? C::kTmemO1 : C::kTmemO0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bd = smem_desc(sv + k * 2048, kBlk128, 1024, kSw128);
+          umma_ts(d, a_t + k * 8, bd, kIdPv, (j >= 2 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_addr(bars, P_PV0 + w));
+        umma_commit(bar_addr(bars, P_VE0 + st));
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0);
+      }
+      if (ok && n_tiles > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < n_tiles) ok = issue_s(j + 2);
+      }
+      if (!ok) {
+        umma_commit(bar_addr(bars, P_DRAIN));
+        drain_wait(bar_addr(bars, P_DRAIN), 0, p.wait_limit_ns, p.status);
+      }
+    }
+  } else {
+    // -------------------------------- softmax ---------------------------------
+    const int qd = warp & 3;
+    const int slot = (warp - 2) >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t t_row = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t s_col = slot ? C::kTmemS1 : C::kTmemS0;
+    const uint32_t o_col = slot ? C::kTmemO1 : C::kTmemO0;
+    const int qi = q0 + r;
+    bool ok = true;
+    if constexpr (kMat) {
+      if (slot == 0) {  // rope block of the query tile: RoPE(q_r) of this row
+        float qr[kDr];
+        rope_query(p, tab, b, qi, h, qr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 w4;
+          w4.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
+          w4.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
+          w4.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
+          w4.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
+          st_sw64_chunk(smem + 2 * kBlk128, r, c, w4);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_addr(bars, P_QR));
+      }
+    }
+    const int n_mine = (n_tiles - slot + 1) / 2;  // tiles slot, slot + 2, ...
+    float m_run = -INFINITY, l_run = 0.0f;
+    for (int i = 0; ok && i < n_mine; ++i) {
+      const int j = 2 * i + slot;
+      if (!warp_wait(bar_addr(bars, P_SF0 + slot), i & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_row + s_col + 32 * c, sr + 32 * c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(sr[e]);
+      }
+      const int64_t kv0 = (int64_t)j * 128;
+      if (kv0 + 128 > p.n_kv) {
+        const int64_t valid = p.n_kv - kv0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = s[c];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      mx[0] = fmaxf(mx[0], mx[4]); mx[1] = fmaxf(mx[1], mx[5]);
+      mx[2] = fmaxf(mx[2], mx[6]); mx[3] = fmaxf(mx[3], mx[7]);
+      mx[0] = fmaxf(mx[0], mx[2]); mx[1] = fmaxf(mx[1], mx[3]);
+      const float m_tile = fmaxf(mx[0], mx[1]) * p.scale_log2;
+      const bool need = m_tile > m_run + 8.0f;
+      const float m_new = need ? m_tile : m_run;
+      const float alpha = fast_exp2(m_run - m_new);
+      float sum[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) sum[c] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = fast_exp2(fmaf(s[64 * c + 2 * e], p.scale_log2, -m_new));
+          const float p1 = fast_exp2(fmaf(s[64 * c + 2 * e + 1], p.scale_log2, -m_new));
+          sum[(2 * e) & 7] += p0;
+          sum[(2 * e + 1) & 7] += p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(t_row + s_col + 32 * c, pk);  // P over the first 64 cells of S_w
+      }
+      sum[0] += sum[4]; sum[1] += sum[5]; sum[2] += sum[6]; sum[3] += sum[7];
+      sum[0] += sum[2]; sum[1] += sum[3];
+      l_run = l_run * alpha + (sum[0] + sum[1]);
+      if (i > 0 && __any_sync(0xffffffffu, need)) {
+        // O_w is rescaled once this slot's previous P.V product has landed (its
+        // next one waits for this tile's P, so the barrier is not ahead of it).
+        if (!warp_wait(bar_addr(bars, P_PV0 + slot), (i - 1) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(t_row + o_col + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(t_row + o_col + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_addr(bars, P_PF0 + slot));
+      m_run = m_new;
+    }
+    // Merge: both slots' last P.V products have landed; each slot writes half of
+    // the output columns from both accumulators.
+    if (ok && n_mine > 0) ok = warp_wait(bar_addr(bars, P_PV0 + slot), (n_mine - 1) & 1, ctl);
+    red[(slot * 2 + 0) * 128 + r] = m_run;
+    red[(slot * 2 + 1) * 128 + r] = l_run;
+    tc_fence_before();
+    mbar_arrive(bar_addr(bars, P_MRG));
+    if (ok) ok = warp_wait(bar_addr(bars, P_MRG), 0, ctl);
+    if (ok) {
+      tc_fence_after();
+      const bool two = n_tiles > 1;  // slot 1 had key tiles (else O_1 was never written)
+      const float m0 = red[r], l0 = red[128 + r];
+      const float m1 = two ? red[256 + r] : -INFINITY, l1 = two ? red[384 + r] : 0.0f;
+      const float m = fmaxf(m0, m1);
+      const float a0 = fast_exp2(m0 - m);
+      const float a1 = two ? fast_exp2(m1 - m) : 0.0f;
+      const float inv_l = 1.0f / (a0 * l0 + a1 * l1);
+      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+      uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int col = 64 * slot + 32 * c;
+        uint32_t v0[32], v1[32];
+        tmem_ld32(t_row + C::kTmemO0 + col, v0);
+        if (two) tmem_ld32(t_row + C::kTmemO1 + col, v1);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x0 = __uint_as_float(v0[2 * e]) * w0, x1 = __uint_as_float(v0[2 * e + 1]) * w0;
+          if (two) {
+            x0 = fmaf(__uint_as_float(v1[2 * e]), w1, x0);
+            x1 = fmaf(__uint_as_float(v1[2 * e + 1]), w1, x1);
+          }
+          pk[e] = pack_bf16x2(x0, x1);
+        }
+        if (qi < p.n_q) {
+          uint4* dst = reinterpret_cast<uint4*>(out_row + col);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_dense_attn(const __grid_constant__ DenseMaps maps, const __grid_constant__ AttnParams p) {
-  attn_body<kKindDense, kDc>(maps, p, nullptr);
+    k_dense_attn(const __grid_constant__ PpMaps maps, const __grid_constant__ AttnParams p) {
+  pp_body<kKindDense>(maps, p, nullptr);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_mat_attn(const __grid_constant__ MatMaps maps, const __grid_constant__ AttnParams p,
-               const __grid_constant__ RopeTable tab) {
-  attn_body<kKindMat, kDc>(maps, p, &tab);
+    k_mat_attn(const __grid_constant__ PpMaps maps, const __grid_constant__ AttnParams p,
+                  const __grid_constant__ RopeTable tab) {
+  pp_body<kKindMat>(maps, p, &tab);
 }
 
 // ---------------------------------------------------------------------------
@@ -993,8 +1252,8 @@ cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, 
                                      int64_t cap, int64_t n_kv, int64_t t0, int grid_h, int grid_w, float scale,
                                      uint16_t* out, int* status, cudaStream_t stream, bool* encode_failed,
                                      const SplitPlan& plan, void* workspace) {
-  using C = Cfg<kKindMla, kDcT>;
-  using L = Layout<kKindMla, kDcT>;
+  using C = Cfg<kDcT>;
+  using L = Layout<kDcT>;
   constexpr int kRow = kDcT + kDr;
   static bool attr_done[64] = {false};
   *encode_failed = false;
@@ -1132,9 +1391,10 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
                                    int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_dense_attn, Layout<kKindDense>::kBytes, attr_done)) return cudaErrorInvalidValue;
-  DenseMaps maps;
-  bool ok = make_head_map(&maps.k, k, batch, n_kv, heads) && make_head_map(&maps.v, v, batch, n_kv, heads);
+  if (!set_smem_attr((const void*)k_dense_attn, PpCfg<kKindDense>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  PpMaps maps;
+  bool ok = make_head_map(&maps.q, q, batch, n_q, heads) && make_head_map(&maps.k, k, batch, n_kv, heads) &&
+            make_head_map(&maps.v, v, batch, n_kv, heads);
   if (!ok) {
     *encode_failed = true;
     return cudaErrorInvalidValue;
@@ -1147,10 +1407,10 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + Cfg<kKindDense>::kBN - 1) / Cfg<kKindDense>::kBN);
+  p.n_kv_tiles = (int)((n_kv + 127) / 128);
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_dense_attn<<<grid, kThreads, Layout<kKindDense>::kBytes, stream>>>(maps, p);
+  k_dense_attn<<<grid, kThreads, PpCfg<kKindDense>::kBytes, stream>>>(maps, p);
   return cudaGetLastError();
 }
 
@@ -1160,13 +1420,14 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
                                  int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_mat_attn, Layout<kKindMat>::kBytes, attr_done)) return cudaErrorInvalidValue;
-  MatMaps maps;
-  bool ok = make_head_map(&maps.k, kv, batch, n_kv, 2 * heads) && make_head_map(&maps.v, kv, batch, n_kv, 2 * heads);
+  if (!set_smem_attr((const void*)k_mat_attn, PpCfg<kKindMat>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  PpMaps maps;
+  bool ok = make_head_map(&maps.q, q, batch, n_q, heads) && make_head_map(&maps.k, kv, batch, n_kv, 2 * heads) &&
+            make_head_map(&maps.v, kv, batch, n_kv, 2 * heads);
   {
     const cuuint64_t dims[3] = {(cuuint64_t)kDrow, (cuuint64_t)n_kv, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)kDrow * 2, (cuuint64_t)cap * kDrow * 2};
-    const cuuint32_t box_r[3] = {32, (cuuint32_t)Cfg<kKindMat>::kBN, 1};
+    const cuuint32_t box_r[3] = {32, 128, 1};
     ok = ok && make_map(&maps.kr, cache, 3, dims, strides, box_r, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (!ok) {
@@ -1182,7 +1443,7 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
   p.n_kv = n_kv;
   p.n_q = n_q;
   p.heads = heads;
-  p.n_kv_tiles = (int)((n_kv + Cfg<kKindMat>::kBN - 1) / Cfg<kKindMat>::kBN);
+  p.n_kv_tiles = (int)((n_kv + 127) / 128);
   p.grid_h = grid_h;
   p.grid_w = grid_w;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -1191,7 +1452,7 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_mat_attn<<<grid, kThreads, Layout<kKindMat>::kBytes, stream>>>(maps, p, tab);
+  k_mat_attn<<<grid, kThreads, PpCfg<kKindMat>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 
