@@ -503,12 +503,21 @@ __device__ __forceinline__ void attn_body(const ChunkMaps& maps, const AttnParam
         umma_commit(bar_addr(bars, B_QABS));
       }
       if (ok) ok = mbar_wait(bar_addr(bars, B_QA), 0, ctl, kDevTimeoutMma);
+      // The issuing thread shares its scheduler with two softmax warps, so it does
+      // as little per MMA as it can: the descriptors of the Qa tile and of ring
+      // stage 0 are built once, and a K step or another stage only moves the start
+      // address (bits [0, 14), 16-byte units; every address here stays below
+      // 2^18).  Ring positions advance as counters.
+      const uint64_t dqa128 = smem_desc(qa, 16, 1024, kSw128), dqa64 = smem_desc(qa, 16, 512, kSw64);
+      const uint64_t dst128 = smem_desc(st0, 16, 1024, kSw128), dst64 = smem_desc(st0, 16, 512, kSw64);
+      const uint64_t dpv = smem_desc(st0, C::kBlkRows, 1024, kSw128);
+      int pst = 0;  // ring stage of the tile whose P.C product is issued next
       auto issue_pv = [&](int jj) -> bool {
         if (!mbar_wait(bar_addr(bars, B_PF0 + (jj & 1)), (jj >> 1) & 1, ctl, kDevTimeoutMma))
           return false;
         tc_fence_after();
         // Value operand: the latent c blocks of the same stage, MN-major.
-        const uint32_t sv = st0 + (jj % kStages) * kStage;
+        const uint64_t dsv = dpv + pst * (kStage >> 4);
         const uint32_t a_t = tmem + ((jj & 1) ? C::kTmemS1 : C::kTmemS0);
         if constexpr (C::kParts == 3) {
           // Two halves of the latent columns; part X of the stage is free after the
@@ -517,31 +526,29 @@ __device__ __forceinline__ void attn_body(const ChunkMaps& maps, const AttnParam
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
 #pragma unroll
-            for (int k = 0; k < kBN / 16; ++k) {
-              const uint64_t bd = smem_desc(sv + half * C::kNbX * C::kBlkRows + k * 2048, C::kBlkRows, 1024, kSw128);
-              umma_ts(tmem + kTmemO + half * 64 * C::kNbX, a_t + k * 8, bd, kIdHalf, (jj > 0 || k > 0) ? 1u : 0u);
-            }
-            if (half == 0) umma_commit(bar_addr(bars, B_KVE0 + kStages + jj % kStages));
+            for (int k = 0; k < kBN / 16; ++k)
+              umma_ts(tmem + kTmemO + half * 64 * C::kNbX, a_t + k * 8,
+                      dsv + ((half * C::kNbX * C::kBlkRows + k * 2048) >> 4), kIdHalf, (jj > 0 || k > 0) ? 1u : 0u);
+            if (half == 0) umma_commit(bar_addr(bars, B_KVE0 + kStages + pst));
           }
           umma_commit(bar_addr(bars, B_PV));
-          umma_commit(bar_addr(bars, B_KVE0 + 2 * kStages + jj % kStages));
+          umma_commit(bar_addr(bars, B_KVE0 + 2 * kStages + pst));
         } else {
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {
-            const uint64_t bd = smem_desc(sv + k * 2048, C::kBlkRows, 1024, kSw128);
-            umma_ts(tmem + kTmemO, a_t + k * 8, bd, kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < kBN / 16; ++k)
+            umma_ts(tmem + kTmemO, a_t + k * 8, dsv + ((k * 2048) >> 4), kIdPv, (jj > 0 || k > 0) ? 1u : 0u);
           umma_commit(bar_addr(bars, B_PV));
-          umma_commit(bar_addr(bars, B_KVE0 + jj % kStages));
+          umma_commit(bar_addr(bars, B_KVE0 + pst));
         }
+        if (++pst == kStages) pst = 0;
         return true;
       };
+      int st = 0, ph = 0;  // ring stage and phase of key tile j
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % kStages;
-        ok = mbar_wait(bar_addr(bars, B_KVF0 + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
+        ok = mbar_wait(bar_addr(bars, B_KVF0 + st), ph, ctl, kDevTimeoutMma);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = st0 + st * kStage;
+        const uint32_t so = st * (kStage >> 4);
         const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
         // S = Qa . [c ; k_r]^T (K = d_c + 32): d_c/16 steps over the 128B-swizzled
         // content blocks, 2 over the 64B-swizzled rope block; Qa and the key tile
@@ -555,19 +562,19 @@ __device__ __forceinline__ void attn_body(const ChunkMaps& maps, const AttnParam
           const int k = C::kParts == 3 ? (n < 2 ? kCs + n : n - 2) : n;
           if (C::kParts == 3 && (n == 2 || n == 2 + kCx)) {  // (part R was waited for above)
             const int x = n == 2 ? 1 : 2;
-            ok = mbar_wait(bar_addr(bars, B_KVF0 + x * kStages + st), (j / kStages) & 1, ctl, kDevTimeoutMma);
+            ok = mbar_wait(bar_addr(bars, B_KVF0 + x * kStages + st), ph, ctl, kDevTimeoutMma);
             if (!ok) break;
             tc_fence_after();
           }
-          const uint32_t off = k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32;
-          const uint32_t sbo = k < kCs ? 1024 : 512;
-          const uint32_t lay = k < kCs ? kSw128 : kSw64;
-          umma_ss(d, smem_desc(qa + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, n > 0);
+          const uint32_t off =
+              (k < kCs ? (k >> 2) * C::kBlkRows + (k & 3) * 32 : C::kNb * C::kBlkRows + (k - kCs) * 32) >> 4;
+          umma_ss(d, (k < kCs ? dqa128 : dqa64) + off, (k < kCs ? dst128 : dst64) + so + off, kIdS, n > 0);
         }
         if (!ok) break;
         if constexpr (C::kParts == 3) umma_commit(bar_addr(bars, B_KVE0 + st));  // R free once S is done
         umma_commit(bar_addr(bars, B_SF0 + (j & 1)));
         if (j >= 1) ok = issue_pv(j - 1);
+        if (++st == kStages) { st = 0; ph ^= 1; }
       }
       if (ok) ok = issue_pv(n_tiles - 1);
       if (ok) {
@@ -959,41 +966,47 @@ __device__ __forceinline__ void pp_body(const PpMaps& maps, const AttnParams& p,
       constexpr uint32_t kIdPv = idesc_bf16_f32(128, kDh, false, true);
       bool ok = mbar_wait(bar_addr(bars, P_Q), 0, ctl, kDevTimeoutMma);
       if (ok && kMat) ok = mbar_wait(bar_addr(bars, P_QR), 0, ctl, kDevTimeoutMma);
-      // S_w = Q . K_j^T (w = j & 1): 8 steps over the 128B-swizzled blocks (+2 over
-      // the 64B-swizzled rope block); the query and key tiles share offsets.
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kKS;
-        if (!mbar_wait(bar_addr(bars, P_KF0 + st), (j / kKS) & 1, ctl, kDevTimeoutMma)) return false;
+      // The issuing thread shares its scheduler with two softmax warps, so it does
+      // as little per MMA as it can: the descriptors of the query tile and of key
+      // and value stage 0 are built once, and a K step or another stage only moves
+      // the start address (bits [0, 14), 16-byte units; every address here stays
+      // below 2^18).  Ring positions advance as counters.
+      const uint64_t dq128 = smem_desc(qs, 16, 1024, kSw128), dq64 = smem_desc(qs, 16, 512, kSw64);
+      const uint64_t dk128 = smem_desc(ks0, 16, 1024, kSw128), dk64 = smem_desc(ks0, 16, 512, kSw64);
+      const uint64_t dv = smem_desc(vs0, kBlk128, 1024, kSw128);
+      int kst = 0, kph = 0, vst = 0, vph = 0;
+      // S_w = Q . K_j^T (w = j & 1) for the next key tile j: 8 steps over the
+      // 128B-swizzled blocks (+2 over the 64B-swizzled rope block); the query and
+      // key tiles share offsets.
+      auto issue_s = [&](int w) -> bool {
+        if (!mbar_wait(bar_addr(bars, P_KF0 + kst), kph, ctl, kDevTimeoutMma)) return false;
         tc_fence_after();
-        const uint32_t sa = ks0 + st * C::kKStage;
-        const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+        const uint32_t so = kst * (C::kKStage >> 4);
+        const uint32_t d = tmem + (w ? C::kTmemS1 : C::kTmemS0);
 #pragma unroll
         for (int k = 0; k < C::kKSteps; ++k) {
-          const uint32_t off = k < 8 ? (k >> 2) * kBlk128 + (k & 3) * 32 : 2 * kBlk128 + (k - 8) * 32;
-          const uint32_t sbo = k < 8 ? 1024 : 512;
-          const uint32_t lay = k < 8 ? kSw128 : kSw64;
-          umma_ss(d, smem_desc(qs + off, 16, sbo, lay), smem_desc(sa + off, 16, sbo, lay), kIdS, k > 0);
+          const uint32_t off = (k < 8 ? (k >> 2) * kBlk128 + (k & 3) * 32 : 2 * kBlk128 + (k - 8) * 32) >> 4;
+          umma_ss(d, (k < 8 ? dq128 : dq64) + off, (k < 8 ? dk128 : dk64) + so + off, kIdS, k > 0);
         }
-        umma_commit(bar_addr(bars, P_SF0 + (j & 1)));
-        umma_commit(bar_addr(bars, P_KE0 + st));
+        umma_commit(bar_addr(bars, P_SF0 + w));
+        umma_commit(bar_addr(bars, P_KE0 + kst));
+        if (++kst == kKS) { kst = 0; kph ^= 1; }
         return true;
       };
       // O_w += P_w . V_j: P from TMEM (bf16 pairs over S_w), V MN-major.
       auto issue_pv = [&](int j) -> bool {
-        const int w = j & 1, st = j % kVS;
+        const int w = j & 1;
         if (!mbar_wait(bar_addr(bars, P_PF0 + w), (j >> 1) & 1, ctl, kDevTimeoutMma)) return false;
-        if (!mbar_wait(bar_addr(bars, P_VF0 + st), (j / kVS) & 1, ctl, kDevTimeoutMma)) return false;
+        if (!mbar_wait(bar_addr(bars, P_VF0 + vst), vph, ctl, kDevTimeoutMma)) return false;
         tc_fence_after();
-        const uint32_t sv = vs0 + st * C::kVStage;
+        const uint64_t dvs = dv + vst * (C::kVStage >> 4);
         const uint32_t a_t = tmem + (w ? C::kTmemS1 : C::kTmemS0);
         const uint32_t d = tmem + (w ? C::kTmemO1 : C::kTmemO0);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(sv + k * 2048, kBlk128, 1024, kSw128);
-          umma_ts(d, a_t + k * 8, bd, kIdPv, (j >= 2 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < 8; ++k) umma_ts(d, a_t + k * 8, dvs + k * (2048 >> 4), kIdPv, (j >= 2 || k > 0) ? 1u : 0u);
         umma_commit(bar_addr(bars, P_PV0 + w));
-        umma_commit(bar_addr(bars, P_VE0 + st));
+        umma_commit(bar_addr(bars, P_VE0 + vst));
+        if (++vst == kVS) { vst = 0; vph ^= 1; }
         return true;
       };
       if (ok) {
@@ -1003,7 +1016,7 @@ __device__ __forceinline__ void pp_body(const PpMaps& maps, const AttnParams& p,
       if (ok && n_tiles > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n_tiles; ++j) {
         ok = issue_pv(j);
-        if (ok && j + 2 < n_tiles) ok = issue_s(j + 2);
+        if (ok && j + 2 < n_tiles) ok = issue_s(j & 1);  // tile j + 2, same slot as j
       }
       if (!ok) {
         umma_commit(bar_addr(bars, P_DRAIN));
