@@ -1189,6 +1189,425 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Two-slot latent kernel for content widths d_c <= 128.  The latent kernel above
+// splits every score tile by columns between its two softmax warpgroups; at
+// d_c <= 128 tensor memory also holds two O_lat accumulators, so here, as in
+// the per-head kernels, softmax warpgroup w owns whole rows of key tiles
+// j = w, w + 2, ... with its own S buffer, O_lat accumulator, max and sum, and
+// the two partial results are merged once before the W_UV epilogue.
+//   [0, 128) S_0 / P_0    [128, 256) S_1 / P_1    [256, 256 + d_c) O_0
+//   [384, 384 + d_c) O_1 (q_abs lands in O_0 first)
+//   epilogue: merged O_lat / l in bf16 at 0 (d_c/2 cells), out accumulator at 128.
+// Keys and values are one ring of [c ; k_r] tiles; a stage is released once its
+// tile's P.C product is done.  The units are those of the latent kernel (heads
+// fastest), without key-range parts.
+// ---------------------------------------------------------------------------
+template <int kDcT>
+struct SlotCfg {
+  static_assert(kDcT == 64 || kDcT == 128, "two-slot latent kernel: d_c 64 or 128");
+  static constexpr int kNb = kDcT / 64;                          // 128B-swizzled content blocks
+  static constexpr uint32_t kStage = kNb * kBlk128 + 128 * 64;   // [c: kNb blocks | k_r: 128 x 64 B]
+  static constexpr int kStages = kDcT == 64 ? 8 : 4;
+  static constexpr int kCs = 4 * kNb;                            // content K steps of the scores
+  static constexpr uint32_t kRingOff = kStage;                   // after the Qa tile
+  static constexpr uint32_t kBarOff = kRingOff + kStages * kStage;
+  static constexpr uint32_t kRedOff = kBarOff + 512;
+  static constexpr uint32_t kUsed = kRedOff + 2 * 2 * 128 * 4;   // (m, l) of both slots
+  static constexpr uint32_t kBytes = kUsed + 1024 <= 232448 ? kUsed + 1024 : 232448;
+  static constexpr uint32_t kMaxPad = kBytes - kUsed;
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
+  static_assert(kUsed + 512 <= 232448, "shared memory (with at least 512 B of alignment slack)");
+  // The prologue parks the q tile (2 blocks) and W_UK_h (kNb blocks) in ring stages 0-1.
+  static_assert((2 + kNb) * kBlk128 <= 2 * kStage && kNb * kBlk128 <= kStage, "prologue operands");
+};
+
+enum SlotBar {
+  L_PRO = 0, L_QABS, L_QA,
+  L_F0, L_E0 = L_F0 + 8,
+  L_SF0 = L_E0 + 8, L_SF1, L_PF0, L_PF1, L_PV0, L_PV1,
+  L_MRG, L_OA, L_OUT, L_DRAIN,
+  L_COUNT
+};
+static_assert(L_COUNT * 8 + 16 <= 512, "barrier area");
+
+template <int kDcT>
+__device__ __forceinline__ void slot_body(const ChunkMaps& maps, const AttnParams& p, const RopeTable* tab) {
+  using C = SlotCfg<kDcT>;
+  constexpr int kS = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
+  const uint32_t pad = (uint32_t)(((raw + 1023) & ~uintptr_t(1023)) - raw);
+  if (pad > C::kMaxPad) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kDevSmemMisaligned);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t qa = smem_u32(smem);      // Qa tile
+  const uint32_t st0 = qa + C::kRingOff;   // ring stage s at st0 + s * kStage
+  const uint32_t bars = qa + C::kBarOff;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * L_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* red = reinterpret_cast<float*>(smem + C::kRedOff);  // [slot][m | l][128 rows]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_qt = (p.n_q + kBM - 1) / kBM;
+  const int unit = (int)blockIdx.x;
+  const int per_b = n_qt * p.heads;
+  const int b = unit / per_b;
+  const int h = (unit % per_b) % p.heads;
+  const int q0 = ((unit % per_b) / p.heads) * kBM;
+  const int n_tiles = p.n_kv_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_addr(bars, L_PRO), 1);
+    mbar_init(bar_addr(bars, L_QABS), 1);
+    mbar_init(bar_addr(bars, L_QA), kSoftmaxThreads);
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(bar_addr(bars, L_F0 + s), 1);
+      mbar_init(bar_addr(bars, L_E0 + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_addr(bars, L_SF0 + s), 1);
+      mbar_init(bar_addr(bars, L_PF0 + s), 128);
+      mbar_init(bar_addr(bars, L_PV0 + s), 1);
+    }
+    mbar_init(bar_addr(bars, L_MRG), kSoftmaxThreads);
+    mbar_init(bar_addr(bars, L_OA), kSoftmaxThreads);
+    mbar_init(bar_addr(bars, L_OUT), 1);
+    mbar_init(bar_addr(bars, L_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------- producer -------------------------------
+      int last_use[kS];
+#pragma unroll
+      for (int s = 0; s < kS; ++s) last_use[s] = -1;
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.wuk);
+      tma_prefetch_desc(&maps.wuv);
+      tma_prefetch_desc(&maps.c);
+      tma_prefetch_desc(&maps.kr);
+      mbar_arrive_expect_tx(bar_addr(bars, L_PRO), (2 + C::kNb) * kBlk128);
+      tma_load_4d(st0, &maps.q, bar_addr(bars, L_PRO), 0, h, q0, b);
+      tma_load_4d(st0 + kBlk128, &maps.q, bar_addr(bars, L_PRO), 64, h, q0, b);
+#pragma unroll
+      for (int i = 0; i < C::kNb; ++i)
+        tma_load_2d(st0 + (2 + i) * kBlk128, &maps.wuk, bar_addr(bars, L_PRO), 64 * i, h * kDh);
+      bool ok = true;
+      int st = 0, use = 0;
+      // n_tiles key tiles, then the W_UV_h blocks as one more ring item.
+      for (int i = 0; ok && i <= n_tiles; ++i) {
+        if (use == 0 && st < 2) ok = mbar_wait(bar_addr(bars, L_QABS), 0, ctl, kDevTimeoutProducer);
+        if (ok && use > 0) ok = mbar_wait(bar_addr(bars, L_E0 + st), (use - 1) & 1, ctl, kDevTimeoutProducer);
+        if (!ok) break;
+        const uint32_t fb = bar_addr(bars, L_F0 + st), sa = st0 + st * C::kStage;
+        if (i < n_tiles) {
+          const int kv0 = i * 128;
+          mbar_arrive_expect_tx(fb, C::kStage);
+          for (int blk = 0; blk < C::kNb; ++blk) tma_load_3d(sa + blk * kBlk128, &maps.c, fb, 64 * blk, kv0, b);
+          tma_load_3d(sa + C::kNb * kBlk128, &maps.kr, fb, kDcT, kv0, b);
+        } else {
+          mbar_arrive_expect_tx(fb, C::kNb * kBlk128);
+          for (int blk = 0; blk < C::kNb; ++blk) tma_load_2d(sa + blk * kBlk128, &maps.wuv, fb, 64 * blk, h * kDh);
+        }
+        last_use[st] = use;
+        if (++st == kS) { st = 0; ++use; }
+      }
+      if (!ok) {
+        drain_wait(bar_addr(bars, L_PRO), 0, p.wait_limit_ns, p.status);
+        for (int s = 0; s < kS; ++s)
+          if (last_use[s] >= 0) drain_wait(bar_addr(bars, L_F0 + s), last_use[s] & 1, p.wait_limit_ns, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------- MMA ----------------------------------
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPv = idesc_bf16_f32(128, kDcT, false, true);
+      bool ok = mbar_wait(bar_addr(bars, L_PRO), 0, ctl, kDevTimeoutMma);
+      if (ok) {
+        tc_fence_after();
+        // q_abs = q_h . W_UK_h (M 128, N d_c, K 128) into O_0: q K-major, W_UK MN-major.
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t a = smem_desc(st0 + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
+          const uint64_t bd = smem_desc(st0 + 2 * kBlk128 + k * 2048, kBlk128, 1024, kSw128);
+          umma_ss(tmem + C::kTmemO0, a, bd, kIdPv, k > 0);
+        }
+        umma_commit(bar_addr(bars, L_QABS));
+      }
+      if (ok) ok = mbar_wait(bar_addr(bars, L_QA), 0, ctl, kDevTimeoutMma);
+      // Descriptors built once; a K step or another stage only moves the start
+      // address (bits [0, 14), 16-byte units; every address here is below 2^18).
+      const uint64_t dqa128 = smem_desc(qa, 16, 1024, kSw128), dqa64 = smem_desc(qa, 16, 512, kSw64);
+      const uint64_t dst128 = smem_desc(st0, 16, 1024, kSw128), dst64 = smem_desc(st0, 16, 512, kSw64);
+      const uint64_t dpv = smem_desc(st0, kBlk128, 1024, kSw128);
+      int sst = 0, sph = 0, pst = 0;  // ring positions of the next score tile and P.C product
+      // S_w = Qa . [c ; k_r]^T for the next key tile (w = its parity).
+      auto issue_s = [&](int w) -> bool {
+        if (!mbar_wait(bar_addr(bars, L_F0 + sst), sph, ctl, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t so = sst * (C::kStage >> 4);
+        const uint32_t d = tmem + (w ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+        for (int k = 0; k < C::kCs + 2; ++k) {
+          const uint32_t off = (k < C::kCs ? (k >> 2) * kBlk128 + (k & 3) * 32 : C::kNb * kBlk128 + (k - C::kCs) * 32) >> 4;
+          umma_ss(d, (k < C::kCs ? dqa128 : dqa64) + off, (k < C::kCs ? dst128 : dst64) + so + off, kIdS, k > 0);
+        }
+        umma_commit(bar_addr(bars, L_SF0 + w));
+        if (++sst == kS) { sst = 0; sph ^= 1; }
+        return true;
+      };
+      // O_w += P_w . C_j: P from TMEM, the latent c blocks of tile j's stage MN-major.
+      auto issue_pv = [&](int j) -> bool {
+        const int w = j & 1;
+        if (!mbar_wait(bar_addr(bars, L_PF0 + w), (j >> 1) & 1, ctl, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint64_t dsv = dpv + pst * (C::kStage >> 4);
+        const uint32_t a_t = tmem + (w ? C::kTmemS1 : C::kTmemS0);
+        const uint32_t d = tmem + (w ? C::kTmemO1 : C::kTmemO0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) umma_ts(d, a_t + k * 8, dsv + k * (2048 >> 4), kIdPv, (j >= 2 || k > 0) ? 1u : 0u);
+        umma_commit(bar_addr(bars, L_PV0 + w));
+        umma_commit(bar_addr(bars, L_E0 + pst));
+        if (++pst == kS) pst = 0;
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0);
+      }
+      if (ok && n_tiles > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        ok = issue_pv(j);
+        if (ok && j + 2 < n_tiles) ok = issue_s(j & 1);  // tile j + 2, same slot as j
+      }
+      if (ok) {
+        // out = O_lat/l . W_UV_h^T (M 128, N 128, K d_c): A from TMEM, W_UV K-major.
+        const int sw = n_tiles % kS;
+        ok = mbar_wait(bar_addr(bars, L_F0 + sw), (n_tiles / kS) & 1, ctl, kDevTimeoutMma) &&
+             mbar_wait(bar_addr(bars, L_OA), 0, ctl, kDevTimeoutMma);
+        if (ok) {
+          tc_fence_after();
+          constexpr uint32_t kIdOut = idesc_bf16_f32(128, 128, false, false);
+          const uint32_t wb = st0 + sw * C::kStage;
+#pragma unroll
+          for (int k = 0; k < kDcT / 16; ++k) {
+            const uint64_t bd = smem_desc(wb + (k >> 2) * kBlk128 + (k & 3) * 32, 16, 1024, kSw128);
+            umma_ts(tmem + C::kTmemS1, tmem + C::kTmemS0 + k * 8, bd, kIdOut, k > 0);
+          }
+          umma_commit(bar_addr(bars, L_OUT));
+        }
+      }
+      if (!ok) {
+        umma_commit(bar_addr(bars, L_DRAIN));
+        drain_wait(bar_addr(bars, L_DRAIN), 0, p.wait_limit_ns, p.status);
+      }
+    }
+  } else {
+    // -------------------------------- softmax ---------------------------------
+    const int qd = warp & 3;
+    const int slot = (warp - 2) >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t t_row = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t s_col = slot ? C::kTmemS1 : C::kTmemS0;
+    const uint32_t o_col = slot ? C::kTmemO1 : C::kTmemO0;
+    const int qi = q0 + r;
+    // q_abs (fp32, O_0) -> bf16 Qa tile in shared memory; this slot converts
+    // latent columns [d_c/2 slot, +d_c/2), the first slot also the rope block.
+    bool ok = warp_wait(bar_addr(bars, L_QABS), 0, ctl);
+    if (ok) {
+      tc_fence_after();
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < C::kNb; ++c) {
+        const int col = (kDcT / 2) * slot + 32 * c;
+        tmem_ld32(t_row + C::kTmemO0 + col, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_sw128_chunk(smem + (col >> 6) * kBlk128, r, ((col & 63) >> 3) + q4, pack8(v + 8 * q4, 1.0f));
+      }
+      if (slot == 0) {
+        float qr[kDr];
+        rope_query(p, tab, b, qi, h, qr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 w4;
+          w4.x = pack_bf16x2(qr[8 * c + 0], qr[8 * c + 1]);
+          w4.y = pack_bf16x2(qr[8 * c + 2], qr[8 * c + 3]);
+          w4.z = pack_bf16x2(qr[8 * c + 4], qr[8 * c + 5]);
+          w4.w = pack_bf16x2(qr[8 * c + 6], qr[8 * c + 7]);
+          st_sw64_chunk(smem + C::kNb * kBlk128, r, c, w4);
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
+      tc_fence_before();
+      mbar_arrive(bar_addr(bars, L_QA));
+    }
+    const int n_mine = (n_tiles - slot + 1) / 2;  // tiles slot, slot + 2, ...
+    float m_run = -INFINITY, l_run = 0.0f;
+    for (int i = 0; ok && i < n_mine; ++i) {
+      const int j = 2 * i + slot;
+      if (!warp_wait(bar_addr(bars, L_SF0 + slot), i & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_row + s_col + 32 * c, sr + 32 * c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(sr[e]);
+      }
+      const int64_t kv0 = (int64_t)j * 128;
+      if (kv0 + 128 > p.n_kv) {
+        const int64_t valid = p.n_kv - kv0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = s[c];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      mx[0] = fmaxf(mx[0], mx[4]); mx[1] = fmaxf(mx[1], mx[5]);
+      mx[2] = fmaxf(mx[2], mx[6]); mx[3] = fmaxf(mx[3], mx[7]);
+      mx[0] = fmaxf(mx[0], mx[2]); mx[1] = fmaxf(mx[1], mx[3]);
+      const float m_tile = fmaxf(mx[0], mx[1]) * p.scale_log2;
+      const bool need = m_tile > m_run + 8.0f;
+      const float m_new = need ? m_tile : m_run;
+      const float alpha = fast_exp2(m_run - m_new);
+      float sum[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) sum[c] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = fast_exp2(fmaf(s[64 * c + 2 * e], p.scale_log2, -m_new));
+          const float p1 = fast_exp2(fmaf(s[64 * c + 2 * e + 1], p.scale_log2, -m_new));
+          sum[(2 * e) & 7] += p0;
+          sum[(2 * e + 1) & 7] += p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(t_row + s_col + 32 * c, pk);  // P over the first 64 cells of S_w
+      }
+      sum[0] += sum[4]; sum[1] += sum[5]; sum[2] += sum[6]; sum[3] += sum[7];
+      sum[0] += sum[2]; sum[1] += sum[3];
+      l_run = l_run * alpha + (sum[0] + sum[1]);
+      if (i > 0 && __any_sync(0xffffffffu, need)) {
+        // O_w is rescaled once this slot's previous P.C product has landed (its
+        // next one waits for this tile's P, so the barrier is not ahead of it).
+        if (!warp_wait(bar_addr(bars, L_PV0 + slot), (i - 1) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < kDcT / 32; ++c) {
+          tmem_ld32(t_row + o_col + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(t_row + o_col + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_addr(bars, L_PF0 + slot));
+      m_run = m_new;
+    }
+    // Merge: both slots' last P.C products have landed; each slot writes half of
+    // the normalised O_lat (bf16, the A operand of the W_UV product) from both
+    // accumulators.
+    if (ok && n_mine > 0) ok = warp_wait(bar_addr(bars, L_PV0 + slot), (n_mine - 1) & 1, ctl);
+    red[(slot * 2 + 0) * 128 + r] = m_run;
+    red[(slot * 2 + 1) * 128 + r] = l_run;
+    tc_fence_before();
+    mbar_arrive(bar_addr(bars, L_MRG));
+    if (ok) ok = warp_wait(bar_addr(bars, L_MRG), 0, ctl);
+    if (ok) {
+      tc_fence_after();
+      const bool two = n_tiles > 1;  // slot 1 had key tiles (else O_1 was never written)
+      const float m0 = red[r], l0 = red[128 + r];
+      const float m1 = two ? red[256 + r] : -INFINITY, l1 = two ? red[384 + r] : 0.0f;
+      const float m = fmaxf(m0, m1);
+      const float a0 = fast_exp2(m0 - m);
+      const float a1 = two ? fast_exp2(m1 - m) : 0.0f;
+      const float inv_l = 1.0f / (a0 * l0 + a1 * l1);
+      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+#pragma unroll
+      for (int c = 0; c < C::kNb; ++c) {
+        const int col = (kDcT / 2) * slot + 32 * c;
+        uint32_t v0[32], v1[32];
+        tmem_ld32(t_row + C::kTmemO0 + col, v0);
+        if (two) tmem_ld32(t_row + C::kTmemO1 + col, v1);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x0 = __uint_as_float(v0[2 * e]) * w0, x1 = __uint_as_float(v0[2 * e + 1]) * w0;
+          if (two) {
+            x0 = fmaf(__uint_as_float(v1[2 * e]), w1, x0);
+            x1 = fmaf(__uint_as_float(v1[2 * e + 1]), w1, x1);
+          }
+          pk[e] = pack_bf16x2(x0, x1);
+        }
+        tmem_st16(t_row + C::kTmemS0 + (kDcT / 4) * slot + 16 * c, pk);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    mbar_arrive(bar_addr(bars, L_OA));
+    if (ok) ok = warp_wait(bar_addr(bars, L_OUT), 0, ctl);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* out_row = p.out + (((int64_t)b * p.n_q + qi) * p.heads + h) * kDh;
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(t_row + C::kTmemS1 + 64 * slot + 32 * c, v);
+        tmem_ld_wait();
+        if (qi < p.n_q) {
+          uint4* dst = reinterpret_cast<uint4*>(out_row + 64 * slot + 32 * c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) dst[q4] = pack8(v + 8 * q4, 1.0f);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int kDcT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_chunk_attn_slots(const __grid_constant__ ChunkMaps maps, const __grid_constant__ AttnParams p,
+                       const __grid_constant__ RopeTable tab) {
+  slot_body<kDcT>(maps, p, &tab);
+}
+
+// ---------------------------------------------------------------------------
 // Host side: tensor maps and launches
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1270,7 +1689,17 @@ cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, 
   constexpr int kRow = kDcT + kDr;
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_chunk_attn<kDcT>, L::kBytes, attr_done)) return cudaErrorInvalidValue;
+  // d_c <= 128 without key-range parts: the two-slot kernel (two O_lat fit in TMEM).
+  constexpr bool kSlots = kDcT <= 128;
+  if (kSlots && plan.split == 1) {
+    if constexpr (kSlots) {
+      static bool slot_attr_done[64] = {false};
+      if (!set_smem_attr((const void*)k_chunk_attn_slots<kDcT>, SlotCfg<kDcT>::kBytes, slot_attr_done))
+        return cudaErrorInvalidValue;
+    }
+  } else if (!set_smem_attr((const void*)k_chunk_attn<kDcT>, L::kBytes, attr_done)) {
+    return cudaErrorInvalidValue;
+  }
   ChunkMaps maps;
   bool ok = make_head_map(&maps.q, q, batch, n_q, heads);
   {
@@ -1322,6 +1751,12 @@ cudaError_t launch_chunk_attention_t(const uint16_t* q, const uint16_t* q_rope, 
   static thread_local RopeTableKey tab_key;
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
+  if constexpr (kSlots) {
+    if (plan.split == 1) {
+      k_chunk_attn_slots<kDcT><<<dim3((unsigned)blocks), kThreads, SlotCfg<kDcT>::kBytes, stream>>>(maps, p, tab);
+      return cudaGetLastError();
+    }
+  }
   k_chunk_attn<kDcT><<<dim3((unsigned)blocks), kThreads, L::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
