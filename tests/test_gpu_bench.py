@@ -40,6 +40,7 @@ def test_bench_tiny_line():
     assert r["traffic"] is None            # the committed ncu summary covers the 480P workload only
     e = b["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert "rotate" in e["l2"]  # no flush inside the end-to-end region: caches rotate past L2
     assert b["gpu_launches"] == 2 * b["steps"]
     a = b["append"]
     assert a["bound"] == "alu" and 0 < a["frac"] < 1.5
