@@ -77,6 +77,39 @@ def test_dc_ragged(vm, d_c):
 
 
 @pytest.mark.parametrize("d_c", DCS)
+def test_dc_ragged_batch(vm, d_c):
+    # three samples with their own seeds and a ragged query and key tile each: the
+    # (sample, query tile, head) decode of every latent kernel
+    w = workload.CONFIGS["tiny"].with_(grid_h=7, grid_w=9, cached_frames=4, heads=3, d_c=d_c, batch=3, seed=78)
+    gc, rc, got, ref = _case(vm, w)
+    assert np.array_equal(gc, rc), f"d_c={d_c}: append not bit-exact"
+    assert_close(got, ref, f"ragged batch 3 d_c={d_c}")
+
+
+@pytest.mark.parametrize("d_c", (64, 128))
+def test_dc_peaked(vm, d_c):
+    # queries and rope queries x4: a peaked softmax that moves the running maximum
+    # often, so the two-slot kernel rescales its accumulators and merges slots whose
+    # maxima differ
+    import torch
+    w = workload.CONFIGS["tiny"].with_(heads=3, d_c=d_c, seed=79)
+    wts = workload.layer_weights(w)
+    act = workload.batch_activations(w)
+    q = workload.bf16_bits(workload.bf16_to_f32(act["q"]) * np.float32(4.0))
+    qr = workload.bf16_bits(workload.bf16_to_f32(act["q_rope"]) * np.float32(4.0))
+    cache = torch.zeros(w.batch, w.n_kv, w.d_c + 32, dtype=torch.bfloat16, device="cuda")
+    _fill(vm, w, to_dev(act["x"]), to_dev(wts["w_dkv"]), to_dev(wts["w_kr"]), cache)
+    out = torch.full((w.batch, w.n_q, w.heads, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_chunk_attention_dc(to_dev(q), to_dev(qr), to_dev(wts["w_uk"]), to_dev(wts["w_uv"]), cache, w.n_kv,
+                               w.chunk_t0, w.grid_h, w.grid_w, SCALE, out)
+    vm.vmla_get_device_status()
+    ref_cache = oracle.cache_append(act["x"], wts["w_dkv"], wts["w_kr"], 0, w.grid_h, w.grid_w)
+    ref = oracle.chunk_attention(q, qr, wts["w_uk"], wts["w_uv"], ref_cache, w.n_kv, w.chunk_t0, w.grid_h,
+                                 w.grid_w, SCALE)
+    assert_close(to_f64(out), ref, f"peaked x4 d_c={d_c}")
+
+
+@pytest.mark.parametrize("d_c", DCS)
 def test_dc_480p_sampled(vm, d_c):
     w = workload.CONFIGS["480p"].with_(d_c=d_c)
     rows = sample_rows(w.n_q, 24, seed=d_c)
