@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stage when its P.V product is.
 // ---------------------------------------------------------------------------
 template <int kKind>
-struct PpCfg {
+struct HeadCfg {
   static constexpr bool kMat = kKind == kKindMat;
   static constexpr int kKSteps = kMat ? 10 : 8;                          // score K steps of 16
   static constexpr uint32_t kQBytes = 2 * kBlk128 + (kMat ? 128u * 64u : 0u);  // q_h (+ rope block)
@@ -828,7 +828,7 @@ struct PpCfg {
   static_assert(kUsed + 512 <= 232448, "shared memory (with at least 512 B of alignment slack)");
 };
 
-enum PpBar {
+enum HeadBar {
   P_Q = 0, P_QR,
   P_KF0, P_KE0 = P_KF0 + 3, P_VF0 = P_KE0 + 3, P_VE0 = P_VF0 + 3,
   P_SF0 = P_VE0 + 3, P_SF1, P_PF0, P_PF1, P_PV0, P_PV1,
@@ -837,7 +837,7 @@ enum PpBar {
 };
 static_assert(P_COUNT * 8 + 16 <= 512, "barrier area");
 
-struct PpMaps {
+struct HeadMaps {
   CUtensorMap q;   // [B, Nq, H, 128] box (64, 1, 128, 1), 128B swizzle
   CUtensorMap k;   // dense: [B, Nk, H, 128]; materialised: [B, n_kv, 2H, 128] (keys at heads [0, H))
   CUtensorMap v;   // dense: [B, Nk, H, 128]; materialised: same tensor (values at head H + h)
@@ -845,8 +845,8 @@ struct PpMaps {
 };
 
 template <int kKind>
-__device__ __forceinline__ void pp_body(const PpMaps& maps, const AttnParams& p, const RopeTable* tab) {
-  using C = PpCfg<kKind>;
+__device__ __forceinline__ void head_body(const HeadMaps& maps, const AttnParams& p, const RopeTable* tab) {
+  using C = HeadCfg<kKind>;
   constexpr bool kMat = C::kMat;
   constexpr int kKS = C::kKStages, kVS = C::kVStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1178,14 +1178,14 @@ __device__ __forceinline__ void pp_body(const PpMaps& maps, const AttnParams& p,
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_dense_attn(const __grid_constant__ PpMaps maps, const __grid_constant__ AttnParams p) {
-  pp_body<kKindDense>(maps, p, nullptr);
+    k_dense_attn(const __grid_constant__ HeadMaps maps, const __grid_constant__ AttnParams p) {
+  head_body<kKindDense>(maps, p, nullptr);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_mat_attn(const __grid_constant__ PpMaps maps, const __grid_constant__ AttnParams p,
-                  const __grid_constant__ RopeTable tab) {
-  pp_body<kKindMat>(maps, p, &tab);
+    k_mat_attn(const __grid_constant__ HeadMaps maps, const __grid_constant__ AttnParams p,
+               const __grid_constant__ RopeTable tab) {
+  head_body<kKindMat>(maps, p, &tab);
 }
 
 // ---------------------------------------------------------------------------
@@ -1458,6 +1458,8 @@ __device__ __forceinline__ void slot_body(const ChunkMaps& maps, const AttnParam
       tc_fence_before();
       mbar_arrive(bar_addr(bars, L_QA));
     }
+    // The per-tile step is the per-head kernels' (written out again: as one shared
+    // inline function it made ptxas spill and measured 0.5-1.8% slower).
     const int n_mine = (n_tiles - slot + 1) / 2;  // tiles slot, slot + 2, ...
     float m_run = -INFINITY, l_run = 0.0f;
     for (int i = 0; ok && i < n_mine; ++i) {
@@ -1839,8 +1841,8 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
                                    int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_dense_attn, PpCfg<kKindDense>::kBytes, attr_done)) return cudaErrorInvalidValue;
-  PpMaps maps;
+  if (!set_smem_attr((const void*)k_dense_attn, HeadCfg<kKindDense>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  HeadMaps maps;
   bool ok = make_head_map(&maps.q, q, batch, n_q, heads) && make_head_map(&maps.k, k, batch, n_kv, heads) &&
             make_head_map(&maps.v, v, batch, n_kv, heads);
   if (!ok) {
@@ -1858,7 +1860,7 @@ cudaError_t launch_dense_attention(const uint16_t* q, const uint16_t* k, const u
   p.n_kv_tiles = (int)((n_kv + 127) / 128);
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_dense_attn<<<grid, kThreads, PpCfg<kKindDense>::kBytes, stream>>>(maps, p);
+  k_dense_attn<<<grid, kThreads, HeadCfg<kKindDense>::kBytes, stream>>>(maps, p);
   return cudaGetLastError();
 }
 
@@ -1868,8 +1870,8 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
                                  int* status, cudaStream_t stream, bool* encode_failed) {
   static bool attr_done[64] = {false};
   *encode_failed = false;
-  if (!set_smem_attr((const void*)k_mat_attn, PpCfg<kKindMat>::kBytes, attr_done)) return cudaErrorInvalidValue;
-  PpMaps maps;
+  if (!set_smem_attr((const void*)k_mat_attn, HeadCfg<kKindMat>::kBytes, attr_done)) return cudaErrorInvalidValue;
+  HeadMaps maps;
   bool ok = make_head_map(&maps.q, q, batch, n_q, heads) && make_head_map(&maps.k, kv, batch, n_kv, 2 * heads) &&
             make_head_map(&maps.v, kv, batch, n_kv, 2 * heads);
   {
@@ -1900,7 +1902,7 @@ cudaError_t launch_mat_attention(const uint16_t* q, const uint16_t* q_rope, cons
   const int per_frame = grid_h * grid_w;
   build_rope_table(&tab, &tab_key, t0, (n_q + per_frame - 1) / per_frame, grid_h, grid_w);
   dim3 grid((unsigned)(((n_q + kBM - 1) / kBM) * heads), (unsigned)batch);
-  k_mat_attn<<<grid, kThreads, PpCfg<kKindMat>::kBytes, stream>>>(maps, p, tab);
+  k_mat_attn<<<grid, kThreads, HeadCfg<kKindMat>::kBytes, stream>>>(maps, p, tab);
   return cudaGetLastError();
 }
 
