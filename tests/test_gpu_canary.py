@@ -97,7 +97,7 @@ def test_canary_attention_forms(vm):
     assert_guards(buf, "dense attention")
 
 
-@pytest.mark.parametrize("d_c", [64, 256])
+@pytest.mark.parametrize("d_c", [64, 128, 256])  # two-slot kernel at 64 and 128
 def test_canary_latent_widths(vm, d_c):
     w = _ragged().with_(d_c=d_c)
     wts = workload.layer_weights(w)
