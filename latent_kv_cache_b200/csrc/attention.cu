@@ -154,6 +154,13 @@ struct AttnParams {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t base, int i) { return base + 8u * i; }
 
+
+// Maximum of three floats in one instruction (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // Bounded wait used when winding down after an abort (ignores the abort flag).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                            int* status) {
@@ -248,13 +255,16 @@ __device__ __forceinline__ bool softmax_tile(int j, int jabs, uint32_t bars, con
   }
   float mx[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) mx[c] = s[c];
+  for (int c = 0; c < 8; ++c) mx[c] = max3f(s[c], s[8 + c], s[16 + c]);
 #pragma unroll
-  for (int c = 8; c < kW; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-  mx[0] = fmaxf(mx[0], mx[4]); mx[1] = fmaxf(mx[1], mx[5]);
-  mx[2] = fmaxf(mx[2], mx[6]); mx[3] = fmaxf(mx[3], mx[7]);
-  mx[0] = fmaxf(mx[0], mx[2]); mx[1] = fmaxf(mx[1], mx[3]);
-  const float lmax = fmaxf(mx[0], mx[1]);
+  for (int c = 24; c < 56; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx[e] = max3f(mx[e], s[c + e], s[c + 8 + e]);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], s[56 + e]);
+  mx[0] = max3f(mx[0], mx[1], mx[2]); mx[3] = max3f(mx[3], mx[4], mx[5]);
+  mx[6] = fmaxf(mx[6], mx[7]);
+  const float lmax = max3f(mx[0], mx[3], mx[6]);
   // The partner's columns of S are read before either half writes P over them.
   float omax;
   if (!exchange(t, bars, j, lmax, omax, ctl)) return false;
@@ -262,23 +272,27 @@ __device__ __forceinline__ bool softmax_tile(int j, int jabs, uint32_t bars, con
   const bool need = m_tile > m_run + 8.0f;
   const float m_new = need ? m_tile : m_run;
   const float alpha = fast_exp2(m_run - m_new);
-  float sum[8];
+  // Pairs of scores in packed fp32x2 instructions (scale-and-subtract, row-sum
+  // accumulators): fewer issue slots for the softmax warps, which share their
+  // schedulers with the MMA-issuing thread.  acc[q] holds the sums of columns
+  // 2e and 2e + 1 with e = q mod 4, the grouping of eight scalar accumulators.
+  float2 acc[4];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) sum[c] = 0.0f;
+  for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.0f, 0.0f);
+  const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-m_new, -m_new);
   uint32_t pk[kW / 2];
 #pragma unroll
   for (int e = 0; e < kW / 2; ++e) {
-    const float p0 = fast_exp2(fmaf(s[2 * e], p.scale_log2, -m_new));
-    const float p1 = fast_exp2(fmaf(s[2 * e + 1], p.scale_log2, -m_new));
-    sum[(2 * e) & 7] += p0;
-    sum[(2 * e + 1) & 7] += p1;
-    pk[e] = pack_bf16x2(p0, p1);
+    const float2 x = __ffma2_rn(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+    const float2 y = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+    acc[e & 3] = __fadd2_rn(acc[e & 3], y);
+    pk[e] = pack_bf16x2(y.x, y.y);
   }
   // P (bf16 pairs) over the first kBN/2 cells of the S buffer: this half's kW/2 cells.
   tmem_st32(t.t_row + sbase + (kW / 2) * t.half, pk);
-  sum[0] += sum[4]; sum[1] += sum[5]; sum[2] += sum[6]; sum[3] += sum[7];
-  sum[0] += sum[2]; sum[1] += sum[3];
-  l_part = l_part * alpha + (sum[0] + sum[1]);
+  acc[0] = __fadd2_rn(acc[0], acc[2]); acc[1] = __fadd2_rn(acc[1], acc[3]);
+  acc[0] = __fadd2_rn(acc[0], acc[1]);
+  l_part = l_part * alpha + (acc[0].x + acc[0].y);
   if (j > 0 && __any_sync(0xffffffffu, need)) {
     // O may only be rescaled once the previous P.C product has landed.  The PV
     // barrier cannot run ahead of PV(j-1) (PV(j) needs this tile's P), so its
