@@ -255,6 +255,23 @@ def test_dense_attention_480p_sampled(vm):
     assert_close(got, ref, "dense 480p")
 
 
+def test_dense_attention_480p_b8_sampled(vm):
+    # eight samples with their own K/V: no cross-sample leakage in the per-head kernel
+    w = workload.CONFIGS["480p_b8"]
+    rows = sample_rows(w.n_q, 64, seed=6)
+    got, ref = _dense_case(vm, w, rows=rows)
+    for b in range(w.batch):
+        assert_close(got[b], ref[b], f"dense 480p b8 sample {b}")
+
+
+def test_dense_attention_1080p_sampled(vm):
+    # 574 key tiles, the last one holding 96 keys
+    w = workload.CONFIGS["1080p"]
+    rows = sample_rows(w.n_q, 128, seed=7)
+    got, ref = _dense_case(vm, w, rows=rows)
+    assert_close(got, ref, "dense 1080p")
+
+
 # ---------------------------------------------------------------------------
 # Failure path: a bounded wait that runs out is reported, and the context survives
 # ---------------------------------------------------------------------------
