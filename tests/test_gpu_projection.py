@@ -172,3 +172,28 @@ def test_projections_minimum_shapes(vm):
     _check(to_f64(q), oracle.linear(x, wq).reshape(1, 1, 1, 128), "q, one token")
     _check(to_f64(qr), oracle.linear(x, wqr).reshape(1, 1, 1, 32), "q_rope, one token")
     _check(to_f64(y), oracle.linear(o.reshape(1, 1, 128), wo), "y, one token")
+
+
+@pytest.mark.parametrize("tokens", [257, 272, 296, 356, 384, 385, 4680 + 256])
+def test_projections_short_last_tile(vm, tokens):
+    """Last M tile of 1, 16, 40, 100, 128, 129 and 72 rows (the pair tile's second
+    CTA holding no rows, or only padding, for the shortest); 3 heads (N = 384 + 96,
+    a partial last column), d_model 256 (query side) and 384 (output side)."""
+    import torch
+    rng = np.random.default_rng(tokens)
+
+    def bits(*shape, std=1.0):
+        return workload.bf16_bits((rng.standard_normal(shape) * std).astype(np.float32))
+
+    H = 3
+    x, wq, wqr = bits(1, tokens, 256), bits(H * 128, 256, std=1 / 16), bits(H * 32, 256, std=1 / 16)
+    q = torch.full((1, tokens, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qr = torch.full((1, tokens, H, 32), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_query_projection(to_dev(x), to_dev(wq), to_dev(wqr), q, qr)
+    o, wo = bits(1, tokens, H, 128), bits(384, H * 128, std=(H * 128) ** -0.5)
+    y = torch.full((1, tokens, 384), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vm.vmla_output_projection(to_dev(o), to_dev(wo), y)
+    vm.vmla_get_device_status()
+    _check(to_f64(q), oracle.linear(x, wq).reshape(1, tokens, H, 128), f"q, {tokens} tokens")
+    _check(to_f64(qr), oracle.linear(x, wqr).reshape(1, tokens, H, 32), f"q_rope, {tokens} tokens")
+    _check(to_f64(y), oracle.linear(o.reshape(1, tokens, H * 128), wo), f"y, {tokens} tokens")
